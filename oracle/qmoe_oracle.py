@@ -1,0 +1,338 @@
+"""Plain CPU oracle of the affine group-quantised MoE gather path.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+Sources, by page and section:
+
+[P1] MLX issue #4509, "gather_qmm at M=1 streams 4-bit expert weights at ~half the
+     bandwidth of M=4 (MoE decode)": the repro script (expert shapes, the SwitchGLU
+     order up, gate, silu(gate)*up, down).
+[P2] MLX PR #4567, "[Metal] Gather mm improvement": Description and Proposed
+     changes (expert-aligned row tiles built from offsets of rhs_indices; the
+     BM = 16, counts 13/8/2/10 example).
+[P3] nuvec-core 0.4.0, tests/quantized.rs: the semantic contract of quantize,
+     dequantize, quantized_matmul and gather_qmm (tests
+     ``round_trip_error_is_about_half_a_step``,
+     ``quantize_snaps_zero_and_handles_constant_and_one_signed_groups``,
+     ``quantized_matmul_equals_the_dequantized_product``,
+     ``gather_qmm_selects_batches``).
+[P5] MTPLX PR #558, "One-kernel MoE combine for Qwen3.5/3.6 MoE prefill on the
+     invariant lane": Summary and Motivation (unsort, weight by the routing
+     scores, sum over top_k, add the gated shared expert).
+
+Conventions.  bf16 tensors are carried as ``uint16`` bit patterns.  Packed codes
+are ``uint32`` words.  Every helper returns fresh arrays and mutates nothing.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "bf16_from_f32", "f32_from_bf16", "pack_codes", "unpack_codes", "quantize",
+    "dequantize", "qmm", "gather_qmm", "sort_by_expert", "tile_table",
+    "silu", "switch_glu", "moe_combine", "sigmoid",
+]
+
+
+# ----------------------------------------------------------------------------- bf16
+
+def f32_from_bf16(u16: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float32 values (exact: bf16 is the top half of fp32)."""
+    u16 = np.asarray(u16, dtype=np.uint16)
+    return (u16.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def bf16_from_f32(f: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest, ties to even; NaN stays a
+    quiet NaN of the same sign."""
+    f = np.ascontiguousarray(np.asarray(f, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    rounded = ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)).astype(np.uint32)
+    nan = np.isnan(f)
+    quiet = ((u >> np.uint64(16)).astype(np.uint32) | np.uint32(0x0040))
+    out = np.where(nan, quiet, rounded)
+    return (out & np.uint32(0xFFFF)).astype(np.uint16)
+
+
+# -------------------------------------------------------------------------- packing
+
+def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
+    """Pack integer codes along the last axis into uint32 words.
+
+    Code j of a word occupies bits [(j mod 32/bits)*bits, ...): the first code of a
+    word sits in its least significant bits.  The packed shape is
+    ``[..., cols*bits/32]`` as in [P3] ``round_trip_error_is_about_half_a_step``.
+    """
+    assert bits in (4, 8)
+    per = 32 // bits
+    codes = np.asarray(codes, dtype=np.uint64)
+    assert codes.shape[-1] % per == 0
+    assert codes.max(initial=0) < (1 << bits)
+    grouped = codes.reshape(codes.shape[:-1] + (codes.shape[-1] // per, per))
+    words = np.zeros(grouped.shape[:-1], dtype=np.uint64)
+    for j in range(per):
+        words |= grouped[..., j] << np.uint64(j * bits)
+    return words.astype(np.uint32)
+
+
+def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
+    """Inverse of :func:`pack_codes`; returns int64 codes."""
+    per = 32 // bits
+    w = np.asarray(words, dtype=np.uint64)
+    mask = np.uint64((1 << bits) - 1)
+    parts = [(w >> np.uint64(j * bits)) & mask for j in range(per)]
+    out = np.stack(parts, axis=-1)
+    return out.reshape(w.shape[:-1] + (w.shape[-1] * per,)).astype(np.int64)
+
+
+# ---------------------------------------------------------------------- quantisation
+
+_EPS = np.float32(1e-7)
+
+
+def quantize(w: np.ndarray, group: int, bits: int, scale_dtype: str = "bf16"):
+    """Affine group quantisation of a 2-D float32 matrix along its last axis.
+
+    Returns ``(packed, scales, biases)``; scales and biases are bf16 bit patterns
+    (``scale_dtype="bf16"``) or float32 (``"f32"``), shape ``[rows, cols/group]``.
+
+    Per group G of ``group`` consecutive values, with n = 2**bits - 1, every
+    operation in float32 and correctly rounded (numpy's float32 arithmetic):
+
+    1. lo = min G, hi = max G; delta = max((hi - lo) / n, 1e-7).
+    2. The edge of larger magnitude is snapped to a code so that zero is exactly
+       representable ([P3] quantize_snaps_zero...): if |lo| > |hi| the edge is lo
+       and the trial step is +delta, otherwise the edge is hi and the step -delta.
+    3. q0 = rint(edge / step).  If q0 != 0 the stored step is edge / q0 and the
+       bias is the edge, so the edge is restored exactly and zero sits on code
+       -q0; snapping can clip the far end of the range by up to one step ([P3]
+       round_trip_error_is_about_half_a_step).  If q0 == 0 the trial step is kept
+       and the bias is 0.
+    4. Step and bias are rounded to the storage type; codes are
+       clamp(rint((w - bias) / step), 0, n) with the STORED step and bias.
+
+    The pages fix the invariants, not these constants (1e-7 floor, the tie rule of
+    step 2, half-even rint, codes from stored values): they are the plainest
+    reading that meets every invariant the pages state.
+    """
+    assert bits in (4, 8) and group in (32, 64, 128)
+    w = np.asarray(w, dtype=np.float32)
+    assert w.ndim == 2 and w.shape[1] % group == 0
+    rows, cols = w.shape
+    n = np.float32((1 << bits) - 1)
+    g = w.reshape(rows, cols // group, group)
+    lo = g.min(axis=-1)
+    hi = g.max(axis=-1)
+    delta = np.maximum((hi - lo) / n, _EPS).astype(np.float32)
+    neg = np.abs(lo) > np.abs(hi)
+    edge = np.where(neg, lo, hi).astype(np.float32)
+    step0 = np.where(neg, delta, -delta).astype(np.float32)
+    q0 = np.rint(edge / step0).astype(np.float32)
+    nz = q0 != 0
+    with np.errstate(divide="ignore", invalid="ignore"):
+        snapped = (edge / np.where(nz, q0, np.float32(1))).astype(np.float32)
+    scale = np.where(nz, snapped, step0).astype(np.float32)
+    bias = np.where(nz, edge, np.float32(0)).astype(np.float32)
+    if scale_dtype == "bf16":
+        s_store, b_store = bf16_from_f32(scale), bf16_from_f32(bias)
+        s_val, b_val = f32_from_bf16(s_store), f32_from_bf16(b_store)
+    elif scale_dtype == "f32":
+        s_store, b_store = scale, bias
+        s_val, b_val = scale, bias
+    else:
+        raise ValueError(scale_dtype)
+    codes = np.rint((g - b_val[..., None]) / s_val[..., None]).astype(np.float32)
+    codes = np.clip(codes, np.float32(0), n).astype(np.int64).reshape(rows, cols)
+    return pack_codes(codes, bits), s_store, b_store
+
+
+def _as_f32(v: np.ndarray) -> np.ndarray:
+    v = np.asarray(v)
+    return f32_from_bf16(v) if v.dtype == np.uint16 else v.astype(np.float32)
+
+
+def dequantize(packed: np.ndarray, scales: np.ndarray, biases: np.ndarray,
+               group: int, bits: int) -> np.ndarray:
+    """w = q*scale + bias per group, in float32 ([P3] ``reference`` helper and
+    round-trip tests).  Leading (expert) dimensions are kept.
+
+    The product is rounded to float32 before the bias is added.  With bf16 scales
+    the product of a <=8-bit code and an 8-bit significand is exact, so this equals
+    a fused multiply-add; with float32 scales it is the two-rounding form.
+    """
+    q = unpack_codes(packed, bits).astype(np.float32)
+    s = _as_f32(scales)
+    b = _as_f32(biases)
+    shp = q.shape
+    qg = q.reshape(shp[:-1] + (shp[-1] // group, group))
+    prod = (qg * s[..., None]).astype(np.float32)
+    return (prod + b[..., None]).astype(np.float32).reshape(shp)
+
+
+# ------------------------------------------------------------------------- matmuls
+
+def qmm(x: np.ndarray, packed, scales, biases, group: int, bits: int) -> np.ndarray:
+    """quantized_matmul with transpose=True: ``x . dequantize(W)^T`` in fp64.
+
+    ``x`` is bf16 bits (uint16) or float; W is ``[N, K*bits/32]``.
+    [P3] quantized_matmul_equals_the_dequantized_product.
+    """
+    xf = _as_f32(x).astype(np.float64)
+    wd = dequantize(packed, scales, biases, group, bits).astype(np.float64)
+    return xf @ wd.T
+
+
+def gather_qmm(x, packed, scales, biases, group: int, bits: int,
+               lhs_indices=None, rhs_indices=None) -> np.ndarray:
+    """gather_qmm with transpose=True ([P3] gather_qmm_selects_batches;
+    [P1] repro script ``gq``).
+
+    ``x``: ``[x_batches, M, K]``; W: ``[E, N, K*bits/32]``.  Batch b of the result
+    is ``x[lhs[b]] . dequantize(W[rhs[b]])^T``.  Missing indices default to every
+    batch in order, x's batch broadcast against the weights'.  Returns fp64
+    ``[B, M, N]``.  Sorted and unsorted index lists take the same path.
+    """
+    x = np.asarray(x)
+    E = packed.shape[0]
+    xb = x.shape[0]
+    if lhs_indices is None and rhs_indices is None:
+        B = max(xb, E)
+        lhs = np.arange(B) % xb if xb == B else np.zeros(B, np.int64)
+        rhs = np.arange(B) % E if E == B else np.zeros(B, np.int64)
+    else:
+        rhs = np.asarray(rhs_indices, np.int64).reshape(-1) if rhs_indices is not None else None
+        lhs = np.asarray(lhs_indices, np.int64).reshape(-1) if lhs_indices is not None else None
+        if lhs is None:
+            B = rhs.size
+            lhs = (np.arange(B) * xb) // B
+        if rhs is None:
+            B = lhs.size
+            rhs = (np.arange(B) * E) // B
+        assert lhs.size == rhs.size
+    wd = dequantize(packed, scales, biases, group, bits).astype(np.float64)
+    xf = _as_f32(x).astype(np.float64)
+    out = np.empty((lhs.size, x.shape[1], packed.shape[1]), np.float64)
+    for b in range(lhs.size):
+        out[b] = xf[lhs[b]] @ wd[rhs[b]].T
+    return out
+
+
+# --------------------------------------------------------------- route metadata
+
+def sort_by_expert(indices: np.ndarray, num_experts: int):
+    """Stable sort of routed rows by expert ([P5] Change: the sorted chain's
+    ``_gather_sort`` and its inverse permutation; [P2] offsets from rhs_indices).
+
+    ``indices``: expert id per routed row r (r = token*top_k + k when flattened).
+    Returns ``order`` (sorted position -> r), ``inv_order`` (r -> sorted position)
+    and ``offsets`` (``[E+1]``, exclusive prefix sums of the per-expert counts).
+    Ties keep ascending r.
+    """
+    keys = np.asarray(indices, np.int64).reshape(-1)
+    assert keys.size == 0 or (keys.min() >= 0 and keys.max() < num_experts)
+    order = np.argsort(keys, kind="stable").astype(np.int64)
+    inv = np.empty_like(order)
+    inv[order] = np.arange(order.size)
+    counts = np.bincount(keys, minlength=num_experts)
+    offsets = np.zeros(num_experts + 1, np.int64)
+    offsets[1:] = np.cumsum(counts)
+    return order, inv, offsets
+
+
+def tile_table(offsets: np.ndarray, bm: int):
+    """Expert-aligned row tiles ([P2] Proposed changes: each tile gets the row to
+    start from, the expert to load and the number of valid rows; no tile spans two
+    experts).
+
+    Experts are visited in order; expert e with c_e rows gets ceil(c_e/bm) tiles
+    starting at offsets[e] + i*bm.  Returns a list of ``(row_start, expert,
+    valid)`` triples.
+    """
+    tiles = []
+    for e in range(len(offsets) - 1):
+        start, end = int(offsets[e]), int(offsets[e + 1])
+        r = start
+        while r < end:
+            tiles.append((r, e, min(bm, end - r)))
+            r += bm
+    return tiles
+
+
+# ------------------------------------------------------------------ MoE blocks
+
+def sigmoid(v):
+    v = np.asarray(v, np.float64)
+    return 1.0 / (1.0 + np.exp(-v))
+
+
+def silu(v):
+    """silu(g) = g * sigmoid(g) ([P1] repro script ``moe``: ``g * mx.sigmoid(g)``)."""
+    v = np.asarray(v, np.float64)
+    return v * sigmoid(v)
+
+
+def switch_glu(x, indices, up, gate, down):
+    """SwitchGLU over routed rows ([P1] repro script ``moe``):
+    u = x.Wup[e]^T, g = x.Wgate[e]^T, h = silu(g)*u, y = h.Wdown[e]^T.
+
+    ``x``: bf16 ``[T, H]``; ``indices``: ``[T, top_k]``; each weight is a tuple
+    ``(packed [E,N,K*bits/32], scales, biases, group, bits)``.  u and g are fp64;
+    h is rounded to bf16 once (it is the bf16 input of the down projection); y is
+    fp64.  Returns ``(y [T, top_k, H], h_bits [T, top_k, I])``.
+    """
+    idx = np.asarray(indices, np.int64)
+    T, top_k = idx.shape
+    xf = _as_f32(x).astype(np.float64)
+
+    def dq(wt):
+        packed, s, b, gs, bits = wt
+        return dequantize(packed, s, b, gs, bits).astype(np.float64)
+
+    wu, wg, wd = dq(up), dq(gate), dq(down)
+    inter = wu.shape[1]
+    hid_out = wd.shape[1]
+    y = np.empty((T, top_k, hid_out), np.float64)
+    h_bits = np.empty((T, top_k, inter), np.uint16)
+    for t in range(T):
+        for k in range(top_k):
+            e = idx[t, k]
+            u = wu[e] @ xf[t]
+            g = wg[e] @ xf[t]
+            h = bf16_from_f32((silu(g) * u).astype(np.float32))
+            h_bits[t, k] = h
+            y[t, k] = wd[e] @ f32_from_bf16(h).astype(np.float64)
+    return y, h_bits
+
+
+def moe_combine(y_sorted, inv_order, scores, shared=None, x=None, w_shared_gate=None):
+    """One-pass MoE combine ([P5] Summary / Motivation):
+
+    out[t] = sum_k scores[t,k] * y_sorted[inv_order[t*top_k + k]]
+             + sigmoid(x[t] . w_shared_gate) * shared[t]
+
+    ``y_sorted``: bf16 ``[T*top_k, H]`` in expert-sorted order; ``scores``: float32
+    ``[T, top_k]``; ``shared``/``x``: bf16 ``[T, H]``; ``w_shared_gate``: bf16
+    ``[H]``.  The shared term is omitted when ``shared`` is None; the gate is 1
+    when ``w_shared_gate`` is None.  Everything in fp64; returns ``[T, H]`` fp64.
+    """
+    ys = _as_f32(y_sorted).astype(np.float64)
+    sc = np.asarray(scores, np.float32).astype(np.float64)
+    T, top_k = sc.shape
+    inv = np.asarray(inv_order, np.int64).reshape(T, top_k)
+    out = np.zeros((T, ys.shape[1]), np.float64)
+    for t in range(T):
+        for k in range(top_k):
+            out[t] += sc[t, k] * ys[inv[t, k]]
+    if shared is not None:
+        sh = _as_f32(shared).astype(np.float64)
+        if w_shared_gate is not None:
+            xf = _as_f32(x).astype(np.float64)
+            wg = _as_f32(w_shared_gate).astype(np.float64)
+            gate = sigmoid(xf @ wg)
+        else:
+            gate = np.ones(T)
+        out += gate[:, None] * sh
+    return out
+
