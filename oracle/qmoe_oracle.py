@@ -211,11 +211,12 @@ def gather_qmm(x, packed, scales, biases, group: int, bits: int,
             B = lhs.size
             rhs = (np.arange(B) * E) // B
         assert lhs.size == rhs.size
-    wd = dequantize(packed, scales, biases, group, bits).astype(np.float64)
     xf = _as_f32(x).astype(np.float64)
     out = np.empty((lhs.size, x.shape[1], packed.shape[1]), np.float64)
-    for b in range(lhs.size):
-        out[b] = xf[lhs[b]] @ wd[rhs[b]].T
+    for e in np.unique(rhs):  # dequantise each selected expert once
+        wd = dequantize(packed[e], scales[e], biases[e], group, bits).astype(np.float64)
+        for b in np.nonzero(rhs == e)[0]:
+            out[b] = xf[lhs[b]] @ wd.T
     return out
 
 
@@ -286,23 +287,22 @@ def switch_glu(x, indices, up, gate, down):
     T, top_k = idx.shape
     xf = _as_f32(x).astype(np.float64)
 
-    def dq(wt):
+    def dq(wt, e):
         packed, s, b, gs, bits = wt
-        return dequantize(packed, s, b, gs, bits).astype(np.float64)
+        return dequantize(packed[e], s[e], b[e], gs, bits).astype(np.float64)
 
-    wu, wg, wd = dq(up), dq(gate), dq(down)
-    inter = wu.shape[1]
-    hid_out = wd.shape[1]
+    inter = up[0].shape[1]
+    hid_out = down[0].shape[1]
     y = np.empty((T, top_k, hid_out), np.float64)
     h_bits = np.empty((T, top_k, inter), np.uint16)
-    for t in range(T):
-        for k in range(top_k):
-            e = idx[t, k]
-            u = wu[e] @ xf[t]
-            g = wg[e] @ xf[t]
+    for e in np.unique(idx):  # dequantise each routed expert once
+        wu, wg, wd = dq(up, e), dq(gate, e), dq(down, e)
+        for t, k in zip(*np.nonzero(idx == e)):
+            u = wu @ xf[t]
+            g = wg @ xf[t]
             h = bf16_from_f32((silu(g) * u).astype(np.float32))
             h_bits[t, k] = h
-            y[t, k] = wd[e] @ f32_from_bf16(h).astype(np.float64)
+            y[t, k] = wd @ f32_from_bf16(h).astype(np.float64)
     return y, h_bits
 
 

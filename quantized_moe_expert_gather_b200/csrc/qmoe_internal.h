@@ -1,0 +1,91 @@
+// Host-side interfaces between the library's translation units.  Not part of the
+// public ABI (include/qmoe.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qmoe.h"
+
+namespace qmoe {
+
+void count_launch(int n = 1);
+int sm_count();
+
+// ----------------------------------------------------------------- quantisation
+cudaError_t launch_quantize(const void* w, bool w_f32, int64_t rows, int64_t cols, int group,
+                            int bits, uint32_t* codes, void* scales, void* biases,
+                            cudaStream_t stream);
+cudaError_t launch_dequantize(const uint32_t* codes, const void* scales, const void* biases,
+                              bool sb_f32, int64_t rows, int64_t cols, int group, int bits,
+                              void* out, bool out_f32, cudaStream_t stream);
+
+// --------------------------------------------------------------- route metadata
+// Routed row r = b*M + m (b in [0, B), m in [0, M)) has expert key rhs(b) and reads
+// x row lhs(b)*M + m, with the NULL-index defaults of qmoe_gather_qmm.
+struct RouteArgs {
+  const uint32_t* rhs = nullptr;   // [B] or null
+  const uint32_t* lhs = nullptr;   // [B] or null
+  int64_t B = 0, M = 1, x_batches = 1, E = 1;
+  int bm = 8;                      // rows per tile of the tile table
+  // outputs (workspace or caller memory)
+  uint32_t* order = nullptr;       // [R]
+  uint32_t* inv_order = nullptr;   // [R]
+  uint32_t* offsets = nullptr;     // [E+1]; offsets[E] = number of valid rows
+  uint32_t* src_row = nullptr;     // [R] x row of each sorted position (nullable)
+  uint32_t* tiles = nullptr;       // [max_tiles*3] (nullable)
+  uint32_t* num_tiles = nullptr;   // [1] (nullable)
+  int64_t max_tiles = 0;
+  // Rows with an invalid index are zeroed in this output: row = by_pos ? sorted
+  // position : r, `zero_cols` bf16 wide.  Nullable.
+  uint16_t* zero_out = nullptr;
+  int64_t zero_cols = 0;
+  bool zero_by_pos = false;
+  int* d_status = nullptr;
+};
+size_t route_workspace_bytes(int64_t R, int64_t E);
+cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream);
+cudaError_t launch_tile_table(const uint32_t* offsets, int64_t E, int bm, uint32_t* tiles,
+                              int64_t max_tiles, uint32_t* num_tiles, int* d_status,
+                              cudaStream_t stream);
+// x_sorted[p] = x[src_row[p]] for p < rows (rows of `cols` bf16).
+cudaError_t launch_gather_rows(const uint16_t* x, const uint32_t* src_row, int64_t rows,
+                               int64_t cols, uint16_t* out, cudaStream_t stream);
+
+// ------------------------------------------------------- gathered quantised matmul
+struct QWeight {
+  const uint32_t* codes;
+  const uint16_t* scales;
+  const uint16_t* biases;
+};
+// One streaming (small rows per expert) or tensor-core (many rows) launch over the
+// expert-aligned tile table.  NMAT = 2 fuses two weight stacks (up, gate) with the
+// silu(gate)*up epilogue.
+struct GemmArgs {
+  QWeight w[2];
+  int nmat = 1;
+  int64_t E = 1, N = 0, K = 0;
+  int group = 64, bits = 4;
+  const uint16_t* x = nullptr;       // activation rows, K wide
+  const uint32_t* src_row = nullptr; // sorted position -> x row (null: identity)
+  uint16_t* y = nullptr;             // output rows, N wide
+  const uint32_t* dst_row = nullptr; // sorted position -> y row (null: identity)
+  const uint32_t* tiles = nullptr;   // (row_start, expert, valid) triples
+  const uint32_t* num_tiles = nullptr;
+  int64_t dense_rows = 0;            // > 0: no tile table, rows [0, dense_rows), expert 0
+  int64_t max_tiles = 0;             // host upper bound of the tile count
+  int bm = 8;                        // rows per tile the table was built with
+  int* d_status = nullptr;
+};
+cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream);   // tiles of <= 16 rows
+cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream); // tiles of 128 rows
+bool qmm_tc_supported(const GemmArgs& a);
+
+// ------------------------------------------------------------------------ combine
+cudaError_t launch_combine(const uint16_t* y_sorted, const uint32_t* inv_order,
+                           const float* scores, const uint16_t* shared, const uint16_t* x,
+                           const uint16_t* w_sg, int64_t T, int top_k, int64_t H, uint16_t* out,
+                           int* d_status, cudaStream_t stream);
+
+}  // namespace qmoe

@@ -1,0 +1,472 @@
+// Streaming gathered quantised matmul for few rows per expert (decode, small M).
+//
+// Computes, for every expert-aligned tile of <= 8*NT routed rows (MLX PR #4567
+// "[Metal] Gather mm improvement", Proposed changes) and every block of 16 output
+// channels, y[row, n] = x[row] . dequantize(W[e])[n]^T (nuvec-core 0.4.0
+// tests/quantized.rs, gather_qmm_selects_batches), and with two weight stacks the
+// SwitchGLU epilogue h = silu(gate) * up (MLX issue #4509 repro script, `moe`).
+//
+// The tile table makes every touched expert's packed weights stream from HBM once
+// per tile (MLX issue #4509: M=1 decode must still reach full bandwidth).
+//
+// Structure (one persistent CTA per SM, 9 warps):
+//   * warp 8 (producer) walks the CTA's contiguous range of (tile, 16-row block)
+//     units and, per K-chunk, loads the 16 packed rows with 2-D TMA boxes of
+//     128 B x 16 rows (128B-swizzled, so the consumers' row-strided reads are free
+//     of bank conflicts) and the matching scales/biases with cp.async, into a ring
+//     of stages guarded by full/empty mbarriers;
+//   * warps 0..7 (consumers) split each chunk's groups.  A lane turns its packed
+//     codes into bf16 "128 + q" (or "2048 + 16*hi" for the high nibble of 8-bit
+//     codes) with one LOP3 per code pair and feeds mma.sync m16n8k16 with W as the
+//     16-row A operand and up to 8 routed rows as the B operand.  Each MMA k-step
+//     stays inside one quantisation group, so per group
+//         sum_k x_k*(q_k*s + b) = s*C + (b - OFFSET*s)*X
+//     with C the MMA sum over the magic-offset codes and X = sum_k x_k, obtained
+//     from one more MMA with an all-ones A.  Scales and biases stay exact (fp32),
+//     accumulation is fp32, and there is one bf16 rounding at the end;
+//   * consumers reduce their partial sums through shared memory and write bf16.
+//
+// All waits are bounded (see qmoe_common.cuh).
+#include <algorithm>
+#include <cstdio>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "qmoe_common.cuh"
+#include "qmoe_internal.h"
+#include "qmoe_tma.h"
+
+namespace qmoe {
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kRows = 16;             // output channels per unit (MMA M)
+constexpr int kSmemBudget = 225 * 1024;
+
+template <int BITS, int GS, int NMAT, int NT>
+struct Cfg {
+  static constexpr int KB_BYTES = GS * BITS / 8;                 // one group of one row
+  static constexpr int CHUNK_ROW_BYTES = std::max(512, KB_BYTES * kConsumerWarps);
+  static constexpr int KB_PER_CHUNK = CHUNK_ROW_BYTES / KB_BYTES;
+  static constexpr int KB_PER_WARP = KB_PER_CHUNK / kConsumerWarps;
+  static constexpr int BOXES = CHUNK_ROW_BYTES / 128;
+  static constexpr int LANE_BYTES = KB_BYTES / 4;                // per row, per lane
+  static constexpr int WORDS = LANE_BYTES / 4;
+  static constexpr int CODE_BYTES = NMAT * BOXES * 2048;
+  static constexpr int SB_BYTES = NMAT * 2 * kRows * KB_PER_CHUNK * 2;
+  static constexpr int STAGE_BYTES = ((CODE_BYTES + SB_BYTES) + 1023) / 1024 * 1024;
+  static constexpr int RED_BYTES = kConsumerWarps * NMAT * NT * kRows * 8 * 4;
+  static constexpr int STAGES =
+      std::min(8, (kSmemBudget - RED_BYTES - 1024) / STAGE_BYTES);
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RED_BYTES + 2 * STAGES * 8 + 64;
+  static constexpr uint32_t TMA_BYTES = CODE_BYTES;
+  static constexpr float OFFSET = BITS == 4 ? 128.0f : 2176.0f;
+  static_assert(STAGES >= 3, "too few pipeline stages");
+  static_assert(KB_PER_WARP >= 1, "chunk smaller than one group per warp");
+};
+
+struct alignas(64) QmvParams {
+  CUtensorMap tmap[2];          // packed codes of each weight stack, [E*N rows, K*bits/32 words]
+  const uint16_t* scales[2];
+  const uint16_t* biases[2];
+  const uint16_t* x;
+  const uint32_t* src_row;
+  const uint32_t* dst_row;
+  uint16_t* y;
+  const uint32_t* tiles;
+  const uint32_t* num_tiles;
+  int64_t dense_rows;
+  int64_t N, K, E;
+  int sb_vec;                   // byte width of the scale/bias copy pieces (2: plain copies)
+  int* d_status;
+};
+
+struct TileInfo {
+  uint32_t row_start, expert, valid;
+};
+
+template <int NT>
+__device__ __forceinline__ TileInfo tile_info(const QmvParams& p, int64_t j) {
+  TileInfo t;
+  if (p.dense_rows > 0) {
+    t.row_start = static_cast<uint32_t>(j * 8 * NT);
+    t.expert = 0;
+    t.valid = static_cast<uint32_t>(imin64(8 * NT, p.dense_rows - j * 8 * NT));
+  } else {
+    t.row_start = p.tiles[3 * j];
+    t.expert = p.tiles[3 * j + 1];
+    t.valid = min(p.tiles[3 * j + 2], static_cast<uint32_t>(8 * NT));
+  }
+  return t;
+}
+
+template <int NT>
+__device__ __forceinline__ int64_t num_tiles(const QmvParams& p) {
+  if (p.dense_rows > 0) return (p.dense_rows + 8 * NT - 1) / (8 * NT);
+  return *p.num_tiles;
+}
+
+// Byte offset of (row, byte c of the chunk row) inside one weight stack's part of a
+// stage: boxes of 16 rows x 128 B, 16-byte chunks XOR-swizzled by (row & 7).
+__device__ __forceinline__ uint32_t swz(int row, int c) {
+  return (c >> 7) * 2048 + row * 128 + ((((c >> 4) & 7) ^ (row & 7)) << 4) + (c & 15);
+}
+
+template <int BITS, int GS, int NMAT, int NT>
+__global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant__ QmvParams p) {
+  using C = Cfg<BITS, GS, NMAT, NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  float* red = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::RED_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1 + 32);                 // producer's expect_tx + 32 cp.async arrivals
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int64_t KB_TOTAL = p.K / GS;
+  const int64_t NCH = (KB_TOTAL + C::KB_PER_CHUNK - 1) / C::KB_PER_CHUNK;
+  const int64_t NB = (p.N + kRows - 1) / kRows;
+  const int64_t units = num_tiles<NT>(p) * NB;
+  const int64_t u_begin = units * blockIdx.x / gridDim.x;
+  const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tmap[0]);
+      if (NMAT > 1) tma_prefetch_desc(&p.tmap[1]);
+    }
+    uint32_t it = 0;
+    bool aborted = false;
+    for (int64_t u = u_begin; u < u_end && !aborted; ++u) {
+      const TileInfo ti = tile_info<NT>(p, u / NB);
+      const int64_t n0 = (u % NB) * kRows;
+      const int64_t row0 = static_cast<int64_t>(ti.expert) * p.N + n0;
+      const int nrows = static_cast<int>(imin64(kRows, p.N - n0));
+      for (int64_t ch = 0; ch < NCH; ++ch, ++it) {
+        const int stage = it % C::STAGES;
+        const uint32_t round = it / C::STAGES;
+        if (round > 0 && !mbar_wait(&empty[stage], (round - 1) & 1, p.d_status)) {
+          *abort_flag = 1;
+        }
+        if (*abort_flag) {
+          aborted = true;
+          break;
+        }
+        uint8_t* st = smem + stage * C::STAGE_BYTES;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], C::TMA_BYTES);
+          const int32_t xw = static_cast<int32_t>(ch * (C::CHUNK_ROW_BYTES / 4));
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+            for (int bx = 0; bx < C::BOXES; ++bx)
+              tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[m], &full[stage], xw + bx * 32,
+                          static_cast<int32_t>(row0));
+        }
+        // scales and biases: [mat][s|b][16 rows][KB_PER_CHUNK] bf16
+        const int64_t kb0 = ch * C::KB_PER_CHUNK;
+        const int ngroups = static_cast<int>(imin64(C::KB_PER_CHUNK, KB_TOTAL - kb0));
+        const int pieces = ngroups * 2 / p.sb_vec;
+        const int tasks = NMAT * 2 * nrows * pieces;
+        uint16_t* sb = reinterpret_cast<uint16_t*>(st + C::CODE_BYTES);
+        for (int tk = lane; tk < tasks; tk += 32) {
+          const int piece = tk % pieces;
+          const int rr = (tk / pieces) % nrows;
+          const int arr = (tk / (pieces * nrows)) % 2;
+          const int m = tk / (pieces * nrows * 2);
+          const uint16_t* src = (arr ? p.biases[m] : p.scales[m]) + (row0 + rr) * KB_TOTAL + kb0;
+          uint16_t* dst = sb + ((m * 2 + arr) * kRows + rr) * C::KB_PER_CHUNK;
+          const int off = piece * (p.sb_vec / 2);
+          if (p.sb_vec == 16)
+            cp_async<16>(dst + off, src + off);
+          else if (p.sb_vec == 8)
+            cp_async<8>(dst + off, src + off);
+          else if (p.sb_vec == 4)
+            cp_async<4>(dst + off, src + off);
+          else
+            dst[off] = src[off];  // odd group count: 2-byte pieces, plain copy
+        }
+        if (p.sb_vec == 2)
+          mbar_arrive(&full[stage]);  // release: orders this lane's plain stores
+        else
+          cp_async_arrive_noinc(&full[stage]);
+      }
+    }
+    if (aborted) {
+      // Let every copy this CTA issued land before the CTA can exit.
+      const uint32_t first = it > static_cast<uint32_t>(C::STAGES) ? it - C::STAGES : 0u;
+      for (uint32_t k = first; k < it; ++k)
+        mbar_wait(&full[k % C::STAGES], (k / C::STAGES) & 1, nullptr);
+    }
+    return;
+  }
+
+  // ----------------------------------------------------------------- consumers
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t ONES = 0x3F803F80u;  // bf16x2 (1, 1)
+  uint32_t it = 0;
+  for (int64_t u = u_begin; u < u_end; ++u) {
+    const TileInfo ti = tile_info<NT>(p, u / NB);
+    const int64_t n0 = (u % NB) * kRows;
+    // x rows of the token slots this lane feeds into the B operand
+    const uint16_t* xrow[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t slot = g + 8 * nt;
+      xrow[nt] = nullptr;
+      if (slot < ti.valid) {
+        const uint32_t pos = ti.row_start + slot;
+        const uint32_t sr = p.src_row ? p.src_row[pos] : pos;
+        xrow[nt] = p.x + static_cast<int64_t>(sr) * p.K;
+      }
+    }
+    float acc[NMAT][NT][4];
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.f;
+
+    for (int64_t ch = 0; ch < NCH; ++ch, ++it) {
+      const int stage = it % C::STAGES;
+      bool ok = false;
+      if (!*abort_flag) {
+        ok = mbar_wait(&full[stage], (it / C::STAGES) & 1, p.d_status);
+        if (!ok) *abort_flag = 1;
+      }
+      if (ok) {
+        const uint8_t* st = smem + stage * C::STAGE_BYTES;
+        const uint16_t* sb = reinterpret_cast<const uint16_t*>(st + C::CODE_BYTES);
+#pragma unroll
+        for (int i = 0; i < C::KB_PER_WARP; ++i) {
+          const int ikb = warp + kConsumerWarps * i;
+          const int64_t kb = ch * C::KB_PER_CHUNK + ikb;
+          if (kb >= KB_TOTAL) break;
+          const int64_t k0 = kb * GS + t * (GS / 4);  // first k of this lane's codes
+          // ---- B operand: x values of this lane's codes, permuted to the MMA k order
+          uint32_t bfr[NT][C::WORDS][2][2];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int j = 0; j < C::WORDS; ++j) {
+              if constexpr (BITS == 4) {
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (xrow[nt]) v = ldg_nc_v4(xrow[nt] + k0 + 8 * j);
+                bfr[nt][j][0][0] = prmt(v.x, v.z, 0x5410);
+                bfr[nt][j][0][1] = prmt(v.x, v.z, 0x7632);
+                bfr[nt][j][1][0] = prmt(v.y, v.w, 0x5410);
+                bfr[nt][j][1][1] = prmt(v.y, v.w, 0x7632);
+              } else {
+                uint2 v = make_uint2(0, 0);
+                if (xrow[nt]) v = ldg_nc_v2(xrow[nt] + k0 + 4 * j);
+                bfr[nt][j][0][0] = prmt(v.x, v.y, 0x5410);
+                bfr[nt][j][0][1] = prmt(v.x, v.y, 0x7632);
+                bfr[nt][j][1][0] = bfr[nt][j][0][0];
+                bfr[nt][j][1][1] = bfr[nt][j][0][1];
+              }
+            }
+          }
+          // ---- X = sum of x over the group (all-ones A operand)
+          float cx[NT][4];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int i2 = 0; i2 < 4; ++i2) cx[nt][i2] = 0.f;
+            const uint32_t ones[4] = {ONES, ONES, ONES, ONES};
+#pragma unroll
+            for (int j = 0; j < C::WORDS; ++j) {
+              mma_bf16_16816(cx[nt], ones, bfr[nt][j][0][0], bfr[nt][j][0][1]);
+              if constexpr (BITS == 4) mma_bf16_16816(cx[nt], ones, bfr[nt][j][1][0], bfr[nt][j][1][1]);
+            }
+          }
+          const int lb = ikb * C::KB_BYTES + t * C::LANE_BYTES;  // lane's byte in the chunk row
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            const uint8_t* cm = st + m * C::BOXES * 2048;
+            uint32_t wg[C::WORDS], wg8[C::WORDS];
+            if constexpr (C::LANE_BYTES == 4) {
+              wg[0] = *reinterpret_cast<const uint32_t*>(cm + swz(g, lb));
+              wg8[0] = *reinterpret_cast<const uint32_t*>(cm + swz(g + 8, lb));
+            } else if constexpr (C::LANE_BYTES == 8) {
+              const uint2 a = *reinterpret_cast<const uint2*>(cm + swz(g, lb));
+              const uint2 b = *reinterpret_cast<const uint2*>(cm + swz(g + 8, lb));
+              wg[0] = a.x; wg[1] = a.y; wg8[0] = b.x; wg8[1] = b.y;
+            } else {
+#pragma unroll
+              for (int q = 0; q < C::LANE_BYTES / 16; ++q) {
+                const uint4 a = *reinterpret_cast<const uint4*>(cm + swz(g, lb + 16 * q));
+                const uint4 b = *reinterpret_cast<const uint4*>(cm + swz(g + 8, lb + 16 * q));
+                wg[4 * q + 0] = a.x; wg[4 * q + 1] = a.y; wg[4 * q + 2] = a.z; wg[4 * q + 3] = a.w;
+                wg8[4 * q + 0] = b.x; wg8[4 * q + 1] = b.y; wg8[4 * q + 2] = b.z; wg8[4 * q + 3] = b.w;
+              }
+            }
+            float cacc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int i2 = 0; i2 < 4; ++i2) cacc[nt][i2] = 0.f;
+#pragma unroll
+            for (int j = 0; j < C::WORDS; ++j) {
+              uint32_t a[2][4];
+              if constexpr (BITS == 4) {
+                const uint32_t M4 = 0x000F000Fu, MAG = 0x43004300u;
+                a[0][0] = and_or(wg[j], M4, MAG);
+                a[0][1] = and_or(wg8[j], M4, MAG);
+                a[0][2] = and_or(wg[j] >> 4, M4, MAG);
+                a[0][3] = and_or(wg8[j] >> 4, M4, MAG);
+                a[1][0] = and_or(wg[j] >> 8, M4, MAG);
+                a[1][1] = and_or(wg8[j] >> 8, M4, MAG);
+                a[1][2] = and_or(wg[j] >> 12, M4, MAG);
+                a[1][3] = and_or(wg8[j] >> 12, M4, MAG);
+              } else {
+                const uint32_t M4 = 0x000F000Fu, LO = 0x43004300u, HI = 0x45004500u;
+                a[0][0] = and_or(wg[j], M4, LO);
+                a[0][1] = and_or(wg8[j], M4, LO);
+                a[0][2] = and_or(wg[j] >> 8, M4, LO);
+                a[0][3] = and_or(wg8[j] >> 8, M4, LO);
+                a[1][0] = and_or(wg[j] >> 4, M4, HI);
+                a[1][1] = and_or(wg8[j] >> 4, M4, HI);
+                a[1][2] = and_or(wg[j] >> 12, M4, HI);
+                a[1][3] = and_or(wg8[j] >> 12, M4, HI);
+              }
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                mma_bf16_16816(cacc[nt], a[0], bfr[nt][j][0][0], bfr[nt][j][0][1]);
+                mma_bf16_16816(cacc[nt], a[1], bfr[nt][j][1][0], bfr[nt][j][1][1]);
+              }
+            }
+            const uint16_t* sm = sb + (m * 2 + 0) * kRows * C::KB_PER_CHUNK + ikb;
+            const uint16_t* bm = sb + (m * 2 + 1) * kRows * C::KB_PER_CHUNK + ikb;
+            const float s0 = bf16_to_f32(sm[g * C::KB_PER_CHUNK]);
+            const float s1 = bf16_to_f32(sm[(g + 8) * C::KB_PER_CHUNK]);
+            const float c0 = fmaf(-C::OFFSET, s0, bf16_to_f32(bm[g * C::KB_PER_CHUNK]));
+            const float c1 = fmaf(-C::OFFSET, s1, bf16_to_f32(bm[(g + 8) * C::KB_PER_CHUNK]));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              acc[m][nt][0] = fmaf(s0, cacc[nt][0], fmaf(c0, cx[nt][0], acc[m][nt][0]));
+              acc[m][nt][1] = fmaf(s0, cacc[nt][1], fmaf(c0, cx[nt][1], acc[m][nt][1]));
+              acc[m][nt][2] = fmaf(s1, cacc[nt][2], fmaf(c1, cx[nt][2], acc[m][nt][2]));
+              acc[m][nt][3] = fmaf(s1, cacc[nt][3], fmaf(c1, cx[nt][3], acc[m][nt][3]));
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+    }
+
+    // ---- cross-warp reduction and epilogue
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float* r = red + (((warp * NMAT + m) * NT + nt) * kRows) * 8;
+        r[g * 8 + 2 * t] = acc[m][nt][0];
+        r[g * 8 + 2 * t + 1] = acc[m][nt][1];
+        r[(g + 8) * 8 + 2 * t] = acc[m][nt][2];
+        r[(g + 8) * 8 + 2 * t + 1] = acc[m][nt][3];
+      }
+    named_bar_sync(1, kConsumerWarps * 32);
+    const int tid = threadIdx.x;
+    if (tid < NT * 128 && !*abort_flag) {
+      const int nt = tid / 128, rem = tid % 128, tok = rem / 16, row = rem % 16;
+      const uint32_t slot = nt * 8 + tok;
+      if (slot < ti.valid && n0 + row < p.N) {
+        float v[NMAT];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          float s = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w)
+            s += red[(((w * NMAT + m) * NT + nt) * kRows + row) * 8 + tok];
+          v[m] = s;
+        }
+        float out = v[0];
+        if constexpr (NMAT == 2) {
+          const float gte = v[1];
+          out = v[0] * (gte / (1.0f + expf(-gte)));
+        }
+        const uint32_t pos = ti.row_start + slot;
+        const uint32_t dr = p.dst_row ? p.dst_row[pos] : pos;
+        p.y[static_cast<int64_t>(dr) * p.N + n0 + row] = f32_to_bf16(out);
+      }
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+  }
+}
+
+template <int BITS, int GS, int NMAT, int NT>
+cudaError_t launch_cfg(const QmvParams& prm, cudaStream_t stream) {
+  using C = Cfg<BITS, GS, NMAT, NT>;
+  auto kern = qmv_kernel<BITS, GS, NMAT, NT>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::SMEM_BYTES + 1024);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<sm_count(), kThreads, C::SMEM_BYTES + 1024, stream>>>(prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int BITS, int GS>
+cudaError_t launch_bits_gs(const QmvParams& prm, int nmat, int nt, cudaStream_t stream) {
+  if (nmat == 2) {
+    return nt == 2 ? launch_cfg<BITS, GS, 2, 2>(prm, stream) : launch_cfg<BITS, GS, 2, 1>(prm, stream);
+  }
+  return nt == 2 ? launch_cfg<BITS, GS, 1, 2>(prm, stream) : launch_cfg<BITS, GS, 1, 1>(prm, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
+  QmvParams prm{};
+  const int64_t words = a.K * a.bits / 32;
+  for (int m = 0; m < a.nmat; ++m) {
+    cudaError_t e = make_tmap_2d_u32(&prm.tmap[m], a.w[m].codes, words, a.E * a.N, 32, 16,
+                                     /*swizzle128=*/true);
+    if (e != cudaSuccess) return e;
+    prm.scales[m] = a.w[m].scales;
+    prm.biases[m] = a.w[m].biases;
+  }
+  prm.x = a.x;
+  prm.src_row = a.src_row;
+  prm.dst_row = a.dst_row;
+  prm.y = a.y;
+  prm.tiles = a.tiles;
+  prm.num_tiles = a.num_tiles;
+  prm.dense_rows = a.dense_rows;
+  prm.N = a.N;
+  prm.K = a.K;
+  prm.E = a.E;
+  const int64_t gpr = a.K / a.group;
+  prm.sb_vec = (gpr % 8 == 0) ? 16 : (gpr % 4 == 0) ? 8 : (gpr % 2 == 0) ? 4 : 2;
+  prm.d_status = a.d_status;
+  const int nt = a.bm > 8 ? 2 : 1;
+  if (a.bits == 4) {
+    if (a.group == 32) return launch_bits_gs<4, 32>(prm, a.nmat, nt, stream);
+    if (a.group == 64) return launch_bits_gs<4, 64>(prm, a.nmat, nt, stream);
+    return launch_bits_gs<4, 128>(prm, a.nmat, nt, stream);
+  }
+  if (a.group == 32) return launch_bits_gs<8, 32>(prm, a.nmat, nt, stream);
+  if (a.group == 64) return launch_bits_gs<8, 64>(prm, a.nmat, nt, stream);
+  return launch_bits_gs<8, 128>(prm, a.nmat, nt, stream);
+}
+
+}  // namespace qmoe

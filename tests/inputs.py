@@ -35,7 +35,7 @@ def random_qweight(rng: np.random.Generator, E: int, N: int, K: int, group: int,
     """Packed codes uniform over [0, 2^bits), bf16 scales ~ U(0.005, 0.02) and
     biases ~ U(-0.1, 0.1).  Codes are drawn as 32-bit words: every bit pattern of a
     word is a valid set of codes, so uniform words give uniform codes."""
-    words = rng.integers(0, 1 << 32, size=(E, N, K * bits // 32), dtype=np.uint64).astype(np.uint32)
+    words = rng.integers(0, 1 << 32, size=(E, N, K * bits // 32), dtype=np.uint32)
     s = bf16_bits(rng.uniform(0.005, 0.02, size=(E, N, K // group)).astype(np.float32))
     b = bf16_bits(rng.uniform(-0.1, 0.1, size=(E, N, K // group)).astype(np.float32))
     return words, s, b

@@ -1,0 +1,268 @@
+"""GPU parity of the floating-point steps against the fp64 oracle:
+|got - want| <= 8e-3 * max|want| for bf16 outputs with fp32 accumulation.
+
+Covers qmm (dense, the decoder-block shapes and the kernel-coverage shapes of
+nuvec-core 0.4.0 tests/quantized.rs), gather_qmm (explicit and default indices,
+sorted and unsorted, bad indices), SwitchGLU (decode and prefill workloads, both
+output modes) and the one-pass combine."""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_util import (assert_close, dev_bf16, dev_f32, dev_u32, host_bits16, host_u32,
+                      qweight, select_experts)
+from inputs import (bf16_bits, decode_tokens, decode_weights, dense_projections,
+                    dense_weight_f32, normal_bf16, prefill_layer, random_qweight, tiny_gather)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=["qmv", "tc"])
+def kernel(request, monkeypatch):
+    monkeypatch.setenv("QMOE_FORCE_KERNEL", request.param)
+    return request.param
+
+
+# ------------------------------------------------------------------------- qmm
+QMM_CASES = [  # (M, N, K, bits, group)
+    (1, 64, 512, 4, 64), (5, 64, 512, 4, 64), (4, 36, 1024, 4, 32), (8, 16, 512, 4, 128),
+    (3, 36, 1024, 4, 32), (1, 13, 96, 8, 32), (4, 24, 256, 8, 128), (40, 64, 256, 4, 64),
+    (33, 50, 128, 8, 32), (64, 96, 4096, 4, 128), (16, 40, 64, 4, 64), (2, 1, 128, 8, 64),
+    (17, 300, 640, 4, 64), (130, 256, 512, 4, 64), (300, 384, 1024, 8, 64),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bits,group", QMM_CASES)
+def test_qmm_matches_oracle(gpu_lib, kernel, M, N, K, bits, group):
+    q = gpu_lib
+    rng = np.random.default_rng(M * 7 + N + K + bits)
+    w, s, b = random_qweight(rng, 1, N, K, group, bits)
+    x = normal_bf16(rng, (M, K))
+    want = O.qmm(x, w[0], s[0], b[0], group, bits)
+    y = q.qmoe_qmm(dev_bf16(x), dev_u32(w[0]), dev_bf16(s[0]), dev_bf16(b[0]), group, bits)
+    torch.cuda.synchronize()
+    assert_close(f"qmm {M}x{N}x{K} {bits}/{group}", y, want)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_qmm_decoder_block_shapes(gpu_lib, bits):
+    """Hidden 2560 projections (q/k/v/o/gate/up/down) at every row count of the
+    small-M benchmark, W = N(0,1)/sqrt(K) quantised on the GPU."""
+    q = gpu_lib
+    rng = np.random.default_rng(bits)
+    for name, N, K in dense_projections():
+        wb16 = bf16_bits(dense_weight_f32(rng, N, K))
+        wc, ws, wb = O.quantize(O.f32_from_bf16(wb16), 64, bits)   # oracle-quantised weights
+        codes, s, b = dev_u32(wc), dev_bf16(ws), dev_bf16(wb)
+        rows = np.arange(0, N, max(1, N // 512))                     # sampled output channels
+        for M in (1, 2, 3, 4, 5, 6, 7, 8, 10, 12, 16):
+            x = normal_bf16(rng, (M, K))
+            y = q.qmoe_qmm(dev_bf16(x), codes, s, b, 64, bits)
+            want = O.qmm(x, wc[rows], ws[rows], wb[rows], 64, bits)
+            assert_close(f"{name} M={M}", y[:, torch.from_numpy(rows).cuda()], want)
+
+
+def test_qmm_few_rows_equal_one_row_bitwise(gpu_lib):
+    """nuvec-core quantized.rs few_row_products_equal_one_row_products_bit_for_bit:
+    each row of a few-row product equals that row's one-row product."""
+    q = gpu_lib
+    rng = np.random.default_rng(1)
+    for M, K, N, group in [(6, 4096, 512, 64), (5, 1024, 1000, 32), (4, 2048, 256, 128)]:
+        w, s, b = random_qweight(rng, 1, N, K, group, 4)
+        x = dev_bf16(normal_bf16(rng, (M, K)))
+        args = (dev_u32(w[0]), dev_bf16(s[0]), dev_bf16(b[0]), group, 4)
+        allr = host_bits16(q.qmoe_qmm(x, *args))
+        for r in range(M):
+            one = host_bits16(q.qmoe_qmm(x[r:r + 1].contiguous(), *args))
+            assert np.array_equal(one[0], allr[r]), (M, K, N, group, r)
+
+
+def test_qmm_empty(gpu_lib):
+    q = gpu_lib
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((16, 8), dtype=torch.int32, device="cuda")
+    s = torch.zeros((16, 1), dtype=torch.bfloat16, device="cuda")
+    y = q.qmoe_qmm(x, w, s, s.clone(), 64, 4)
+    assert tuple(y.shape) == (0, 16)
+
+
+# ------------------------------------------------------------------- gather_qmm
+def test_tiny_gather_sorted_and_unsorted(gpu_lib, kernel):
+    q = gpu_lib
+    d = tiny_gather(0)
+    T, K = d["x"].shape
+    x3 = d["x"].reshape(T, 1, K)
+    rhs = d["idx"].reshape(-1)
+    want = O.gather_qmm(x3, d["w"], d["s"], d["b"], d["group"], d["bits"], None, rhs)
+    args = (dev_u32(d["w"]), dev_bf16(d["s"]), dev_bf16(d["b"]))
+    y = q.qmoe_gather_qmm(dev_bf16(x3), *args, None, dev_u32(rhs), d["group"], d["bits"])
+    assert_close("tiny unsorted", y.reshape(T, 2, -1), want.reshape(T, 2, -1))
+    perm = np.argsort(rhs, kind="stable")
+    lhs = (np.arange(rhs.size) // 2)[perm].astype(np.uint32)
+    ys = q.qmoe_gather_qmm(dev_bf16(x3), *args, dev_u32(lhs), dev_u32(rhs[perm]), d["group"],
+                           d["bits"], sorted_indices=True)
+    assert np.array_equal(host_bits16(ys), host_bits16(y)[perm])
+
+
+GATHER_CASES = [  # (E, N, K, M, batches, sorted, bits, group)
+    (8, 64, 512, 1, 6, False, 4, 64), (8, 36, 192, 1, 5, False, 4, 32),
+    (4, 64, 256, 40, 3, False, 4, 64), (4, 40, 128, 33, 2, False, 8, 32),
+    (8, 64, 256, 1, 100, True, 4, 64), (8, 64, 256, 1, 20, True, 8, 128),
+    (16, 48, 192, 1, 70, True, 4, 32), (32, 128, 1024, 2, 300, False, 4, 64),
+]
+
+
+@pytest.mark.parametrize("E,N,K,M,batches,sorted_,bits,group", GATHER_CASES)
+def test_gather_qmm_matches_oracle(gpu_lib, kernel, E, N, K, M, batches, sorted_, bits, group):
+    q = gpu_lib
+    rng = np.random.default_rng(E + N + K + M + batches)
+    w, s, b = random_qweight(rng, E, N, K, group, bits)
+    x = normal_bf16(rng, (batches, M, K))
+    ids = np.array([(i * 7 + 3) % E for i in range(batches)], np.uint32)
+    if sorted_:
+        ids.sort()
+    want = O.gather_qmm(x, w, s, b, group, bits, None, ids)
+    y = q.qmoe_gather_qmm(dev_bf16(x), dev_u32(w), dev_bf16(s), dev_bf16(b), None, dev_u32(ids),
+                          group, bits, sorted_indices=sorted_)
+    assert_close("gather", y, want)
+
+
+def test_gather_qmm_explicit_and_default_indices(gpu_lib):
+    q = gpu_lib
+    rng = np.random.default_rng(0x71)
+    E, N, K, group, bits = 3, 8, 64, 32, 4
+    w, s, b = random_qweight(rng, E, N, K, group, bits)
+    x = normal_bf16(rng, (4, 2, K))
+    lhs, rhs = np.array([3, 0, 2], np.uint32), np.array([1, 2, 0], np.uint32)
+    args = (dev_u32(w), dev_bf16(s), dev_bf16(b))
+    y = q.qmoe_gather_qmm(dev_bf16(x), *args, dev_u32(lhs), dev_u32(rhs), group, bits)
+    assert_close("explicit", y, O.gather_qmm(x, w, s, b, group, bits, lhs, rhs))
+    x1 = x[:1, :1]
+    y = q.qmoe_gather_qmm(dev_bf16(x1), *args, None, None, group, bits)
+    assert_close("default", y, O.gather_qmm(x1, w, s, b, group, bits))
+
+
+def test_gather_qmm_bad_indices_zero_rows(gpu_lib):
+    q = gpu_lib
+    rng = np.random.default_rng(5)
+    E, N, K, group, bits = 4, 32, 128, 64, 4
+    w, s, b = random_qweight(rng, E, N, K, group, bits)
+    x = normal_bf16(rng, (3, 1, K))
+    rhs = np.array([1, 7, 2, 0, 3, 9], np.uint32)  # 7 and 9 are out of range
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q.qmoe_gather_qmm(dev_bf16(x), dev_u32(w), dev_bf16(s), dev_bf16(b), None, dev_u32(rhs),
+                          group, bits, status=status)
+    got = y.float().cpu().numpy()
+    ok = rhs < E
+    want = O.gather_qmm(x, w, s, b, group, bits, np.arange(6) // 2, np.where(ok, rhs, 0))
+    assert np.all(got[~ok] == 0)
+    assert_close("valid rows", y[torch.from_numpy(ok).cuda()], want[ok])
+    assert int(status.item()) & q.QMOE_DEV_BAD_INDEX
+
+
+# ------------------------------------------------------------------- switch_glu
+def _switch_oracle(x, idx, up, gate, down, group, bits):
+    experts = np.unique(idx)
+    remap = np.searchsorted(experts, idx)
+    sel = lambda wt: (*select_experts(wt, experts), group, bits)
+    return O.switch_glu(x, remap, sel(up), sel(gate), sel(down))
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_switch_glu_decode_layer(gpu_lib, M):
+    """Decode layer at full size: hidden 4096, intermediate 2048, E=288, top-8."""
+    q = gpu_lib
+    up, gate, down = _decode_weights()
+    x, idx = decode_tokens(0, M)
+    W = [qweight(*t, 64, 4) for t in (up, gate, down)]
+    y = q.qmoe_switch_glu(dev_bf16(x), dev_u32(idx), *W, mode=0)
+    want, _ = _switch_oracle(x, idx, up, gate, down, 64, 4)
+    assert_close(f"decode M={M}", y, want)
+
+
+_DECODE = {}
+
+
+def _decode_weights():
+    if "w" not in _DECODE:
+        _DECODE["w"] = decode_weights(0)
+    return _DECODE["w"]
+
+
+@pytest.mark.parametrize("T,mode", [(64, 0), (512, 1), (713, 0)])
+def test_switch_glu_prefill(gpu_lib, kernel, T, mode):
+    """Prefill SwitchGLU with Zipf-skewed routing (hidden 2048, intermediate 512,
+    E=256, top-8), token-order and expert-sorted outputs."""
+    q = gpu_lib
+    d = _prefill(T)
+    W = [qweight(*d[k], 64, 4) for k in ("up", "gate", "down")]
+    want, _ = _switch_oracle(d["x"], d["idx"], d["up"], d["gate"], d["down"], 64, 4)
+    if mode == 0:
+        y = q.qmoe_switch_glu(dev_bf16(d["x"]), dev_u32(d["idx"]), *W, mode=0)
+        assert_close(f"prefill T={T}", y, want)
+    else:
+        ys, inv = q.qmoe_switch_glu(dev_bf16(d["x"]), dev_u32(d["idx"]), *W, mode=1)
+        inv = host_u32(inv)
+        _, w_inv, _ = O.sort_by_expert(d["idx"].reshape(-1), d["E"])
+        assert np.array_equal(inv, w_inv)
+        assert_close(f"prefill sorted T={T}", ys[torch.from_numpy(inv.astype(np.int64)).cuda()],
+                     want.reshape(T * d["top_k"], -1))
+
+
+_PREFILL = {}
+
+
+def _prefill(T):
+    if T not in _PREFILL:
+        _PREFILL[T] = prefill_layer(0, T)
+    return _PREFILL[T]
+
+
+# --------------------------------------------------------------------- combine
+@pytest.mark.parametrize("T", [128, 331])
+@pytest.mark.parametrize("gated", [True, False])
+def test_moe_combine(gpu_lib, T, gated):
+    q = gpu_lib
+    rng = np.random.default_rng(T)
+    K, H, E = 8, 2048, 256
+    keys = rng.integers(0, E, size=T * K)
+    order, inv, _ = O.sort_by_expert(keys, E)
+    y_sorted = normal_bf16(rng, (T * K, H))
+    scores = rng.random((T, K)).astype(np.float32) / K
+    shared = normal_bf16(rng, (T, H))
+    x = normal_bf16(rng, (T, H))
+    wsg = normal_bf16(rng, (H,), 1 / np.sqrt(H))
+    want = O.moe_combine(y_sorted, inv, scores, shared, x if gated else None,
+                         wsg if gated else None)
+    out = q.qmoe_moe_combine(dev_bf16(y_sorted), dev_u32(inv.astype(np.uint32)), dev_f32(scores),
+                             dev_bf16(shared), dev_bf16(x) if gated else None,
+                             dev_bf16(wsg) if gated else None)
+    assert_close(f"combine T={T}", out, want)
+
+
+def test_moe_block_prefill_with_shared_expert(gpu_lib):
+    """MoE block: routed experts in expert order + shared SwiGLU + sigmoid gate, one
+    combine pass (T = 128)."""
+    q = gpu_lib
+    T = 128
+    d = prefill_layer(1, T, shared=True)
+    W = [qweight(*d[k], 64, 4) for k in ("up", "gate", "down")]
+    S = [qweight(*d[k], 64, 4) for k in ("sh_up", "sh_gate", "sh_down")]
+    xd = dev_bf16(d["x"])
+    ys, inv = q.qmoe_switch_glu(xd, dev_u32(d["idx"]), *W, mode=1)
+    zeros = torch.zeros((T, 1), dtype=torch.int32, device="cuda")
+    sh = q.qmoe_switch_glu(xd, zeros, *S, mode=0).reshape(T, -1)
+    out = q.qmoe_moe_combine(ys, inv, dev_f32(d["scores"]), sh, xd, dev_bf16(d["w_sg"]))
+    # oracle chain: its own bf16 expert outputs and shared output feed its combine
+    y_tok, _ = _switch_oracle(d["x"], d["idx"], d["up"], d["gate"], d["down"], 64, 4)
+    sh_want, _ = O.switch_glu(d["x"], np.zeros((T, 1), np.int64),
+                              (*d["sh_up"], 64, 4), (*d["sh_gate"], 64, 4), (*d["sh_down"], 64, 4))
+    order, w_inv, _ = O.sort_by_expert(d["idx"].reshape(-1), d["E"])
+    y_sorted = O.bf16_from_f32(y_tok.reshape(T * d["top_k"], -1)[order].astype(np.float32))
+    sh_b = O.bf16_from_f32(sh_want[:, 0].astype(np.float32))
+    want = O.moe_combine(y_sorted, w_inv, d["scores"], sh_b, d["x"], d["w_sg"])
+    assert_close("moe block", out, want)
