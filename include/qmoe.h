@@ -83,6 +83,18 @@ QMOE_API const char* qmoe_status_string(int status);
 QMOE_API uint64_t qmoe_launch_count(void);
 
 /*
+ * Kernel timing (benchmark instrumentation).  While enabled, every kernel launch of
+ * the library is bracketed by two CUDA events recorded on its stream, keyed by the
+ * kernel's name ("route", "gather_rows", "qmv", "qmv_glu", "tc", "tc_glu",
+ * "combine", "quantize", "dequantize").  qmoe_timing_enable(1) clears earlier
+ * records; qmoe_timing_read() waits for the recorded events of one kernel name and
+ * returns their summed elapsed time and launch count (0 launches if none).  Host
+ * state only; returns QMOE_ERR_CUDA if an event call fails.
+ */
+QMOE_API int qmoe_timing_enable(int on);
+QMOE_API int qmoe_timing_read(const char* kernel, double* total_ms, uint64_t* launches);
+
+/*
  * qmoe_quantize -- affine group quantisation along the last axis ([P3]
  * round_trip_error_is_about_half_a_step, quantize_snaps_zero_and_handles_constant_
  * and_one_signed_groups).

@@ -19,7 +19,7 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "QmoeError", "load", "library_path", "qmoe_status_string", "qmoe_launch_count",
+    "QmoeError", "load", "library_path", "qmoe_status_string", "qmoe_launch_count", "qmoe_timing_enable", "qmoe_timing_read",
     "qmoe_quantize", "qmoe_dequantize", "qmoe_qmm", "qmoe_gather_qmm",
     "qmoe_gather_qmm_workspace_size", "qmoe_sort_by_expert", "qmoe_tile_table",
     "qmoe_switch_glu", "qmoe_switch_glu_workspace_size", "qmoe_moe_combine", "QWeight",
@@ -47,6 +47,9 @@ class _QWeight(ctypes.Structure):
 _SIGS = {
     "qmoe_status_string": (ctypes.c_char_p, [_i32]),
     "qmoe_launch_count": (ctypes.c_uint64, []),
+    "qmoe_timing_enable": (_i32, [_i32]),
+    "qmoe_timing_read": (_i32, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
+                                ctypes.POINTER(ctypes.c_uint64)]),
     "qmoe_quantize": (_i32, [_p, _i32, _i64, _i64, _i32, _i32, _p, _p, _p, _p]),
     "qmoe_dequantize": (_i32, [_p, _p, _p, _i32, _i64, _i64, _i32, _i32, _p, _i32, _p]),
     "qmoe_qmm": (_i32, [_p, _i64, _p, _p, _p, _i64, _i64, _i32, _i32, _p, _p, _p]),
@@ -130,6 +133,20 @@ def qmoe_status_string(status: int) -> str:
 
 def qmoe_launch_count() -> int:
     return int(load().qmoe_launch_count())
+
+
+def qmoe_timing_enable(on: bool) -> None:
+    """Record CUDA events around every library kernel launch (clears old records)."""
+    _check("qmoe_timing_enable", load().qmoe_timing_enable(int(bool(on))))
+
+
+def qmoe_timing_read(kernel: str):
+    """``(total_ms, launches)`` of the recorded launches of one kernel name."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_uint64(0)
+    _check("qmoe_timing_read", load().qmoe_timing_read(kernel.encode(), ctypes.byref(ms),
+                                                       ctypes.byref(n)))
+    return ms.value, int(n.value)
 
 
 def qmoe_quantize(w: torch.Tensor, group: int = 64, bits: int = 4):

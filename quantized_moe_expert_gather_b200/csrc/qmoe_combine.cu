@@ -96,6 +96,7 @@ cudaError_t launch_combine(const uint16_t* y_sorted, const uint32_t* inv_order,
                            const uint16_t* w_sg, int64_t T, int top_k, int64_t H, uint16_t* out,
                            int* d_status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
+  LaunchTimer timer("combine", stream);
   combine_kernel<<<static_cast<unsigned>(T), kThreads, 0, stream>>>(
       y_sorted, inv_order, scores, shared, x, w_sg, T, top_k, H, out, d_status);
   count_launch();

@@ -13,6 +13,22 @@ namespace qmoe {
 void count_launch(int n = 1);
 int sm_count();
 
+// Brackets one kernel launch with timing events while qmoe_timing_enable(1) is in
+// effect (otherwise free).  Construct it right before the launch; it records the
+// stop event when it goes out of scope.
+class LaunchTimer {
+ public:
+  LaunchTimer(const char* kernel, cudaStream_t stream);
+  ~LaunchTimer();
+  LaunchTimer(const LaunchTimer&) = delete;
+  LaunchTimer& operator=(const LaunchTimer&) = delete;
+
+ private:
+  const char* name_;
+  cudaStream_t stream_;
+  void* start_ = nullptr;
+};
+
 // ----------------------------------------------------------------- quantisation
 cudaError_t launch_quantize(const void* w, bool w_f32, int64_t rows, int64_t cols, int group,
                             int bits, uint32_t* codes, void* scales, void* biases,

@@ -420,6 +420,7 @@ cudaError_t launch_cfg(const QmvParams& prm, cudaStream_t stream) {
                                     C::SMEM_BYTES + 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  LaunchTimer timer(NMAT == 2 ? "qmv_glu" : "qmv", stream);
   kern<<<sm_count(), kThreads, C::SMEM_BYTES + 1024, stream>>>(prm);
   count_launch();
   return cudaGetLastError();

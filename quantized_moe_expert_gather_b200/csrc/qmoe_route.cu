@@ -273,6 +273,7 @@ cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream) {
     cudaFuncSetAttribute(route_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(cnt_bytes));
   }
+  LaunchTimer timer("route", stream);
   if (nchunks <= 1) {
     route_fused_kernel<<<1, kChunk, cnt_bytes, stream>>>(d);
     count_launch();
@@ -288,6 +289,7 @@ cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream) {
 cudaError_t launch_tile_table(const uint32_t* offsets, int64_t E, int bm, uint32_t* tiles,
                               int64_t max_tiles, uint32_t* num_tiles, int* d_status,
                               cudaStream_t stream) {
+  LaunchTimer timer("route", stream);
   tile_table_kernel<<<1, kChunk, 0, stream>>>(offsets, E, bm, tiles, max_tiles, num_tiles,
                                                d_status);
   count_launch();
@@ -300,6 +302,7 @@ cudaError_t launch_gather_rows(const uint16_t* x, const uint32_t* src_row, int64
   const int64_t n = rows * (cols / 8);
   const int threads = 256;
   const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 16);
+  LaunchTimer timer("gather_rows", stream);
   gather_rows_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, src_row, rows,
                                                                             cols, out);
   count_launch();

@@ -83,6 +83,14 @@ def decode_tokens(seed: int, M: int, H=4096, E=288, top_k=8):
     return x, idx
 
 
+def decode_scores(seed: int, M: int, top_k=8):
+    """Positive combine weights per token summing to 1 (the decode repro has no
+    router; any normalised scores serve the combine)."""
+    rng = np.random.default_rng(2000 + seed)
+    w = rng.random((M, top_k)).astype(np.float32) + np.float32(0.05)
+    return (w / w.sum(axis=1, keepdims=True)).astype(np.float32)
+
+
 DENSE = dict(hidden=2560, q_out=4096, kv_out=1024, inter=9728, layers=36, sets=8)
 
 
