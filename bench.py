@@ -346,7 +346,8 @@ def main():
     ms_per_step = ms_max / args.steps
 
     # instrumented graph: CUDA events captured around every kernel of the step
-    q.qmoe_timing_enable(True)
+    slots = torch.zeros(16 * 4 * LAYERS * 4, dtype=torch.uint8, device=dev)
+    q.qmoe_timing_enable(slots)
     g_timed, _ = capture()
     sums = {k: 0.0 for k in ("qmv_glu", "qmv", "route", "combine")}
     counts = {k: 0 for k in sums}
@@ -360,7 +361,7 @@ def main():
             sums[k] += t
             counts[k] += n
         ug_bytes += sum(touched[s * LAYERS + l] for l in range(LAYERS)) * UPGATE_BYTES
-    q.qmoe_timing_enable(False)
+    q.qmoe_timing_enable(None)
     del g_timed
     k_ms, k_n = sums["qmv_glu"], counts["qmv_glu"]
     peaks = measured_peaks()

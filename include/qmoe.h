@@ -83,15 +83,21 @@ QMOE_API const char* qmoe_status_string(int status);
 QMOE_API uint64_t qmoe_launch_count(void);
 
 /*
- * Kernel timing (benchmark instrumentation).  While enabled, every kernel launch of
- * the library is bracketed by two CUDA events recorded on its stream, keyed by the
- * kernel's name ("route", "gather_rows", "qmv", "qmv_glu", "tc", "tc_glu",
- * "combine", "quantize", "dequantize").  qmoe_timing_enable(1) clears earlier
- * records; qmoe_timing_read() waits for the recorded events of one kernel name and
- * returns their summed elapsed time and launch count (0 launches if none).  Host
- * state only; returns QMOE_ERR_CUDA if an event call fails.
+ * Kernel timing (benchmark instrumentation, works inside CUDA graphs).
+ *   qmoe_timing_enable(slots, capacity): from now on every kernel launch of the
+ *     library takes the next of `capacity` 16-byte slots of the caller's DEVICE
+ *     buffer `slots`, zeroes it in stream order and records in it the earliest CTA
+ *     start and the latest CTA end (the GPU's global nanosecond timer), keyed on the
+ *     host by the kernel's name ("route", "gather_rows", "qmv", "qmv_glu", "tc",
+ *     "tc_glu", "combine").  Launches beyond `capacity` are not timed.  Earlier
+ *     records are cleared.  slots = NULL turns timing off.
+ *   qmoe_timing_read(kernel, &ms, &n): copies the slots back (synchronously: call it
+ *     after the timed work has finished) and returns the summed durations and the
+ *     number of timed launches of that kernel name.  Replaying a captured graph
+ *     rewrites the same slots, so read after each replay.
+ * Returns QMOE_ERR_ARG for a null output pointer, QMOE_ERR_CUDA if the copy fails.
  */
-QMOE_API int qmoe_timing_enable(int on);
+QMOE_API int qmoe_timing_enable(void* slots, int64_t capacity);
 QMOE_API int qmoe_timing_read(const char* kernel, double* total_ms, uint64_t* launches);
 
 /*

@@ -47,7 +47,7 @@ class _QWeight(ctypes.Structure):
 _SIGS = {
     "qmoe_status_string": (ctypes.c_char_p, [_i32]),
     "qmoe_launch_count": (ctypes.c_uint64, []),
-    "qmoe_timing_enable": (_i32, [_i32]),
+    "qmoe_timing_enable": (_i32, [_p, _i64]),
     "qmoe_timing_read": (_i32, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
                                 ctypes.POINTER(ctypes.c_uint64)]),
     "qmoe_quantize": (_i32, [_p, _i32, _i64, _i64, _i32, _i32, _p, _p, _p, _p]),
@@ -135,9 +135,14 @@ def qmoe_launch_count() -> int:
     return int(load().qmoe_launch_count())
 
 
-def qmoe_timing_enable(on: bool) -> None:
-    """Record CUDA events around every library kernel launch (clears old records)."""
-    _check("qmoe_timing_enable", load().qmoe_timing_enable(int(bool(on))))
+def qmoe_timing_enable(slots: Optional[torch.Tensor]) -> None:
+    """Time every following library kernel launch into ``slots`` (a CUDA uint8
+    tensor of 16 bytes per launch); ``None`` turns timing off."""
+    if slots is None:
+        _check("qmoe_timing_enable", load().qmoe_timing_enable(None, 0))
+        return
+    _need(slots, "slots", (torch.uint8,))
+    _check("qmoe_timing_enable", load().qmoe_timing_enable(_ptr(slots), slots.numel() // 16))
 
 
 def qmoe_timing_read(kernel: str):

@@ -30,11 +30,12 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
     const uint16_t* __restrict__ y_sorted, const uint32_t* __restrict__ inv_order,
     const float* __restrict__ scores, const uint16_t* __restrict__ shared,
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ w_sg, int64_t T, int top_k,
-    int64_t H, uint16_t* __restrict__ out, int* d_status) {
+    int64_t H, uint16_t* __restrict__ out, int* d_status, ProfSlot* prof) {
   __shared__ float red[kThreads / 32];
   __shared__ float gate_sh;
   const int64_t t = blockIdx.x;
   const int tid = threadIdx.x;
+  if (tid == 0) prof_start(prof);
   const int64_t nvec = H / 8;
   const int64_t R = T * top_k;
 
@@ -87,6 +88,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
     o.w = pack_bf16x2(acc[6], acc[7]);
     reinterpret_cast<uint4*>(out + t * H)[v] = o;
   }
+  __syncthreads();
+  if (tid == 0) prof_end(prof);
 }
 
 }  // namespace
@@ -98,7 +101,7 @@ cudaError_t launch_combine(const uint16_t* y_sorted, const uint32_t* inv_order,
   if (T == 0) return cudaSuccess;
   LaunchTimer timer("combine", stream);
   combine_kernel<<<static_cast<unsigned>(T), kThreads, 0, stream>>>(
-      y_sorted, inv_order, scores, shared, x, w_sg, T, top_k, H, out, d_status);
+      y_sorted, inv_order, scores, shared, x, w_sg, T, top_k, H, out, d_status, timer.slot());
   count_launch();
   return cudaGetLastError();
 }

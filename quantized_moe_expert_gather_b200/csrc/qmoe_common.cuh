@@ -35,6 +35,22 @@ __device__ __forceinline__ void set_status(int* d_status, int bits) {
   if (d_status != nullptr) atomicOr(d_status, bits);
 }
 
+// -------------------------------------------------------------- launch timing
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Call from one thread per CTA at its start / after its last work.
+template <typename Slot>
+__device__ __forceinline__ void prof_start(Slot* p) {
+  if (p != nullptr) atomicMax(&p->start_inv, ~global_ns());
+}
+template <typename Slot>
+__device__ __forceinline__ void prof_end(Slot* p) {
+  if (p != nullptr) atomicMax(&p->end, global_ns());
+}
+
 // ------------------------------------------------------------------- mbarriers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -51,27 +51,9 @@ void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
 namespace {
 struct TimingState {
   std::mutex mu;
-  bool on = false;
-  std::vector<cudaEvent_t> pool;  // free events
-  std::map<std::string, std::vector<std::pair<cudaEvent_t, cudaEvent_t>>> recs;
-  cudaEvent_t take() {
-    if (!pool.empty()) {
-      cudaEvent_t e = pool.back();
-      pool.pop_back();
-      return e;
-    }
-    cudaEvent_t e = nullptr;
-    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
-    return e;
-  }
-  void clear() {
-    for (auto& kv : recs)
-      for (auto& pr : kv.second) {
-        pool.push_back(pr.first);
-        pool.push_back(pr.second);
-      }
-    recs.clear();
-  }
+  ProfSlot* slots = nullptr;
+  int64_t capacity = 0;
+  std::vector<std::string> names;  // kernel name of each used slot
 };
 TimingState& timing() {
   static TimingState* t = new TimingState();  // never destroyed: safe at process exit
@@ -79,45 +61,14 @@ TimingState& timing() {
 }
 }  // namespace
 
-LaunchTimer::LaunchTimer(const char* kernel, cudaStream_t stream) : name_(kernel), stream_(stream) {
+LaunchTimer::LaunchTimer(const char* kernel, cudaStream_t stream) {
   TimingState& t = timing();
   std::lock_guard<std::mutex> g(t.mu);
-  if (!t.on) return;
-  cudaEvent_t e = t.take();
-  if (e != nullptr && cudaEventRecord(e, stream_) == cudaSuccess) start_ = e;
-}
-
-LaunchTimer::~LaunchTimer() {
-  if (start_ == nullptr) return;
-  TimingState& t = timing();
-  std::lock_guard<std::mutex> g(t.mu);
-  cudaEvent_t e = t.take();
-  if (e != nullptr && cudaEventRecord(e, stream_) == cudaSuccess)
-    t.recs[name_].emplace_back(static_cast<cudaEvent_t>(start_), e);
-}
-
-int sm_count() {
-  static int cache[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (cache[dev] == 0) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 1;
-  }
-  return cache[dev];
-}
-
-cudaError_t make_tmap_2d_u32(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
-                             int box_inner, int box_rows, bool swizzle128) {
-  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, base, inner, rows, box_inner,
-                   box_rows, swizzle128);
-}
-cudaError_t make_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
-                              int box_inner, int box_rows, bool swizzle128) {
-  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, rows, box_inner,
-                   box_rows, swizzle128);
+  if (t.slots == nullptr || static_cast<int64_t>(t.names.size()) >= t.capacity) return;
+  ProfSlot* s = t.slots + t.names.size();
+  if (cudaMemsetAsync(s, 0, sizeof(ProfSlot), stream) != cudaSuccess) return;
+  t.names.emplace_back(kernel);
+  slot_ = s;
 }
 
 }  // namespace qmoe
@@ -126,11 +77,12 @@ extern "C" {
 
 uint64_t qmoe_launch_count(void) { return qmoe::g_launches.load(); }
 
-int qmoe_timing_enable(int on) {
+int qmoe_timing_enable(void* slots, int64_t capacity) {
   auto& t = qmoe::timing();
   std::lock_guard<std::mutex> g(t.mu);
-  if (on) t.clear();
-  t.on = on != 0;
+  t.names.clear();
+  t.slots = capacity > 0 ? static_cast<qmoe::ProfSlot*>(slots) : nullptr;
+  t.capacity = t.slots ? capacity : 0;
   return QMOE_OK;
 }
 
@@ -140,13 +92,16 @@ int qmoe_timing_read(const char* kernel, double* total_ms, uint64_t* launches) {
   std::lock_guard<std::mutex> g(t.mu);
   *total_ms = 0.0;
   *launches = 0;
-  auto it = t.recs.find(kernel);
-  if (it == t.recs.end()) return QMOE_OK;
-  for (auto& pr : it->second) {
-    if (cudaEventSynchronize(pr.second) != cudaSuccess) return QMOE_ERR_CUDA;
-    float ms = 0.f;
-    if (cudaEventElapsedTime(&ms, pr.first, pr.second) != cudaSuccess) return QMOE_ERR_CUDA;
-    *total_ms += ms;
+  if (t.slots == nullptr || t.names.empty()) return QMOE_OK;
+  std::vector<qmoe::ProfSlot> host(t.names.size());
+  if (cudaMemcpy(host.data(), t.slots, host.size() * sizeof(qmoe::ProfSlot),
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return QMOE_ERR_CUDA;
+  for (size_t i = 0; i < host.size(); ++i) {
+    if (t.names[i] != kernel || host[i].end == 0 || host[i].start_inv == 0) continue;
+    const unsigned long long start = ~host[i].start_inv;
+    if (host[i].end < start) continue;
+    *total_ms += static_cast<double>(host[i].end - start) * 1e-6;
     *launches += 1;
   }
   return QMOE_OK;

@@ -13,20 +13,23 @@ namespace qmoe {
 void count_launch(int n = 1);
 int sm_count();
 
-// Brackets one kernel launch with timing events while qmoe_timing_enable(1) is in
-// effect (otherwise free).  Construct it right before the launch; it records the
-// stop event when it goes out of scope.
+// Device-side timing record of one launch: ~(earliest CTA start) and the latest
+// CTA end, in global-timer nanoseconds, both combined with atomicMax.
+struct ProfSlot {
+  unsigned long long start_inv;
+  unsigned long long end;
+};
+
+// While qmoe_timing_enable() is in effect, reserves the next timing slot for one
+// launch of `kernel` and zeroes it on `stream`; slot() is null otherwise.  Pass
+// slot() to the kernel.
 class LaunchTimer {
  public:
   LaunchTimer(const char* kernel, cudaStream_t stream);
-  ~LaunchTimer();
-  LaunchTimer(const LaunchTimer&) = delete;
-  LaunchTimer& operator=(const LaunchTimer&) = delete;
+  ProfSlot* slot() const { return slot_; }
 
  private:
-  const char* name_;
-  cudaStream_t stream_;
-  void* start_ = nullptr;
+  ProfSlot* slot_ = nullptr;
 };
 
 // ----------------------------------------------------------------- quantisation

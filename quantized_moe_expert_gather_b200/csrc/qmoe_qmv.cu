@@ -80,6 +80,7 @@ struct alignas(64) QmvParams {
   int64_t N, K, E;
   int sb_vec;                   // byte width of the scale/bias copy pieces (2: plain copies)
   int* d_status;
+  ProfSlot* prof;
 };
 
 struct TileInfo {
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
     }
     *abort_flag = 0;
     fence_mbar_init();
+    prof_start(p.prof);
   }
   __syncthreads();
 
@@ -407,10 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
     }
     named_bar_sync(1, kConsumerWarps * 32);
   }
+  if (threadIdx.x == 0) prof_end(p.prof);
 }
 
 template <int BITS, int GS, int NMAT, int NT>
-cudaError_t launch_cfg(const QmvParams& prm, cudaStream_t stream) {
+cudaError_t launch_cfg(QmvParams prm, cudaStream_t stream) {
   using C = Cfg<BITS, GS, NMAT, NT>;
   auto kern = qmv_kernel<BITS, GS, NMAT, NT>;
   static std::once_flag once;
@@ -421,6 +424,7 @@ cudaError_t launch_cfg(const QmvParams& prm, cudaStream_t stream) {
   });
   if (attr_err != cudaSuccess) return attr_err;
   LaunchTimer timer(NMAT == 2 ? "qmv_glu" : "qmv", stream);
+  prm.prof = timer.slot();
   kern<<<sm_count(), kThreads, C::SMEM_BYTES + 1024, stream>>>(prm);
   count_launch();
   return cudaGetLastError();

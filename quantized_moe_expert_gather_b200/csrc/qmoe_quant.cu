@@ -121,7 +121,6 @@ cudaError_t launch_quantize(const void* w, bool w_f32, int64_t rows, int64_t col
   if (n == 0) return cudaSuccess;
   const int threads = 128;
   const unsigned blocks = static_cast<unsigned>((n + threads - 1) / threads);
-  LaunchTimer timer("quantize", stream);
   if (w_f32) {
     auto* wp = static_cast<const float*>(w);
     auto* sp = static_cast<float*>(scales);
@@ -165,7 +164,6 @@ cudaError_t launch_dequantize(const uint32_t* codes, const void* scales, const v
                               bool sb_f32, int64_t rows, int64_t cols, int group, int bits,
                               void* out, bool out_f32, cudaStream_t stream) {
   if (rows * cols == 0) return cudaSuccess;
-  LaunchTimer timer("dequantize", stream);
   if (sb_f32 && out_f32)
     dequant_dispatch<float, float>(codes, scales, biases, rows, cols, group, bits, out, stream);
   else if (sb_f32)

@@ -41,6 +41,7 @@ struct RouteDev {
   int64_t zero_cols;
   bool zero_by_pos;
   int* d_status;
+  ProfSlot* prof;
 };
 
 // Expert key of routed row r (E for an invalid expert or x row) and its x row.
@@ -170,42 +171,55 @@ __device__ void phase_scan(const RouteDev& d, int64_t nchunks, uint32_t* sh) {
 __device__ void phase_scatter(const RouteDev& d, int64_t chunk) {
   const int64_t nb = d.E + 1;
   const int64_t r = chunk * kChunk + threadIdx.x;
-  if (r >= d.R) return;
-  uint32_t xrow;
-  const uint32_t key = row_key(d, r, &xrow);
-  const uint32_t pos = d.hist[chunk * nb + key] + d.lrank[r];
-  d.order[pos] = static_cast<uint32_t>(r);
-  d.inv_order[r] = pos;
-  if (d.src_row) d.src_row[pos] = xrow;
-  if (key == static_cast<uint32_t>(d.E)) set_status(d.d_status, QMOE_DEV_BAD_INDEX);
-  if (key == static_cast<uint32_t>(d.E) && d.zero_out != nullptr) {
-    const int64_t row = d.zero_by_pos ? static_cast<int64_t>(pos) : r;
-    uint16_t* dst = d.zero_out + row * d.zero_cols;
-    for (int64_t c = 0; c < d.zero_cols; ++c) dst[c] = 0;
+  if (r < d.R) {
+    uint32_t xrow;
+    const uint32_t key = row_key(d, r, &xrow);
+    const uint32_t pos = d.hist[chunk * nb + key] + d.lrank[r];
+    d.order[pos] = static_cast<uint32_t>(r);
+    d.inv_order[r] = pos;
+    if (d.src_row) d.src_row[pos] = xrow;
+    if (key == static_cast<uint32_t>(d.E)) set_status(d.d_status, QMOE_DEV_BAD_INDEX);
+    if (key == static_cast<uint32_t>(d.E) && d.zero_out != nullptr) {
+      const int64_t row = d.zero_by_pos ? static_cast<int64_t>(pos) : r;
+      uint16_t* dst = d.zero_out + row * d.zero_cols;
+      for (int64_t c = 0; c < d.zero_cols; ++c) dst[c] = 0;
+    }
   }
 }
 
 __global__ void __launch_bounds__(kChunk) route_count_kernel(RouteDev d) {
   extern __shared__ uint8_t cnt[];
+  if (threadIdx.x == 0) prof_start(d.prof);
   phase_count(d, blockIdx.x, cnt);
+  __syncthreads();
+  if (threadIdx.x == 0) prof_end(d.prof);
 }
 __global__ void __launch_bounds__(kChunk) route_scan_kernel(RouteDev d, int64_t nchunks) {
   __shared__ uint32_t sh[32];
+  if (threadIdx.x == 0) prof_start(d.prof);
   phase_scan(d, nchunks, sh);
+  __syncthreads();
+  if (threadIdx.x == 0) prof_end(d.prof);
 }
 __global__ void __launch_bounds__(kChunk) route_scatter_kernel(RouteDev d) {
+  if (threadIdx.x == 0) prof_start(d.prof);
   phase_scatter(d, blockIdx.x);
+  __syncthreads();
+  if (threadIdx.x == 0) prof_end(d.prof);
 }
 // R <= 1024: all three phases in one CTA.  Global writes of one phase are read by
 // other threads of the same CTA after __syncthreads.
 __global__ void __launch_bounds__(kChunk) route_fused_kernel(RouteDev d) {
   extern __shared__ uint8_t cnt[];
   __shared__ uint32_t sh[32];
+  if (threadIdx.x == 0) prof_start(d.prof);
   phase_count(d, 0, cnt);
   __syncthreads();
   phase_scan(d, 1, sh);
   __syncthreads();
   phase_scatter(d, 0);
+  __syncthreads();
+  if (threadIdx.x == 0) prof_end(d.prof);
 }
 __global__ void __launch_bounds__(kChunk)
     tile_table_kernel(const uint32_t* offsets, int64_t E, int bm, uint32_t* tiles,
@@ -216,7 +230,8 @@ __global__ void __launch_bounds__(kChunk)
 
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x,
                                    const uint32_t* __restrict__ src_row, int64_t rows,
-                                   int64_t cols, uint16_t* __restrict__ out) {
+                                   int64_t cols, uint16_t* __restrict__ out, ProfSlot* prof) {
+  if (threadIdx.x == 0) prof_start(prof);
   // cols is a multiple of 8: 16-byte vectors.
   const int64_t vec_per_row = cols / 8;
   const int64_t n = rows * vec_per_row;
@@ -227,6 +242,8 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x,
     reinterpret_cast<uint4*>(out + p * cols)[v] =
         reinterpret_cast<const uint4*>(x + sr * cols)[v];
   }
+  __syncthreads();
+  if (threadIdx.x == 0) prof_end(prof);
 }
 
 inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
@@ -273,14 +290,27 @@ cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream) {
     cudaFuncSetAttribute(route_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(cnt_bytes));
   }
-  LaunchTimer timer("route", stream);
   if (nchunks <= 1) {
+    LaunchTimer timer("route", stream);
+    d.prof = timer.slot();
     route_fused_kernel<<<1, kChunk, cnt_bytes, stream>>>(d);
     count_launch();
   } else {
-    route_count_kernel<<<static_cast<unsigned>(nchunks), kChunk, cnt_bytes, stream>>>(d);
-    route_scan_kernel<<<1, kChunk, 0, stream>>>(d, nchunks);
-    route_scatter_kernel<<<static_cast<unsigned>(nchunks), kChunk, 0, stream>>>(d);
+    {
+      LaunchTimer timer("route", stream);
+      d.prof = timer.slot();
+      route_count_kernel<<<static_cast<unsigned>(nchunks), kChunk, cnt_bytes, stream>>>(d);
+    }
+    {
+      LaunchTimer timer("route", stream);
+      d.prof = timer.slot();
+      route_scan_kernel<<<1, kChunk, 0, stream>>>(d, nchunks);
+    }
+    {
+      LaunchTimer timer("route", stream);
+      d.prof = timer.slot();
+      route_scatter_kernel<<<static_cast<unsigned>(nchunks), kChunk, 0, stream>>>(d);
+    }
     count_launch(3);
   }
   return cudaGetLastError();
@@ -289,7 +319,6 @@ cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream) {
 cudaError_t launch_tile_table(const uint32_t* offsets, int64_t E, int bm, uint32_t* tiles,
                               int64_t max_tiles, uint32_t* num_tiles, int* d_status,
                               cudaStream_t stream) {
-  LaunchTimer timer("route", stream);
   tile_table_kernel<<<1, kChunk, 0, stream>>>(offsets, E, bm, tiles, max_tiles, num_tiles,
                                                d_status);
   count_launch();
@@ -304,7 +333,7 @@ cudaError_t launch_gather_rows(const uint16_t* x, const uint32_t* src_row, int64
   const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 16);
   LaunchTimer timer("gather_rows", stream);
   gather_rows_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, src_row, rows,
-                                                                            cols, out);
+                                                                            cols, out, timer.slot());
   count_launch();
   return cudaGetLastError();
 }

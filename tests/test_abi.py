@@ -36,6 +36,14 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(raw, n), n
 
 
+def test_timing_hook_off_without_gpu(lib):
+    assert lib.qmoe_timing_enable(None, 0) == 0
+    ms, n = ctypes.c_double(1.0), ctypes.c_uint64(7)
+    assert lib.qmoe_timing_read(b"qmv", ctypes.byref(ms), ctypes.byref(n)) == 0
+    assert ms.value == 0.0 and n.value == 0
+    assert lib.qmoe_timing_read(b"qmv", None, None) == ERR_ARG
+
+
 def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4, -5):
         assert q.qmoe_status_string(s).startswith("QMOE_")

@@ -1,0 +1,41 @@
+"""The device-side launch timing hook records one slot per launch, eagerly and
+inside a captured CUDA graph."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import dev_bf16, dev_u32
+from inputs import normal_bf16, random_qweight
+
+pytestmark = pytest.mark.gpu
+
+
+def test_timing_slots_eager_and_graph(gpu_lib):
+    q = gpu_lib
+    rng = np.random.default_rng(0)
+    w, s, b = random_qweight(rng, 1, 4096, 4096, 64, 4)
+    args = (dev_u32(w[0]), dev_bf16(s[0]), dev_bf16(b[0]), 64, 4)
+    x = dev_bf16(normal_bf16(rng, (4, 4096)))
+    y = torch.empty((4, 4096), dtype=torch.bfloat16, device="cuda")
+    slots = torch.zeros(16 * 8, dtype=torch.uint8, device="cuda")
+    q.qmoe_qmm(x, *args, out=y)          # eager warm-up outside timing
+    torch.cuda.synchronize()
+    q.qmoe_timing_enable(slots)
+    try:
+        q.qmoe_qmm(x, *args, out=y)
+        torch.cuda.synchronize()
+        ms, n = q.qmoe_timing_read("qmv")
+        assert n == 1 and 0.0 < ms < 50.0
+        assert q.qmoe_timing_read("combine") == (0.0, 0)
+        q.qmoe_timing_enable(slots)       # clears the records
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            q.qmoe_qmm(x, *args, out=y)
+        for _ in range(2):
+            g.replay()
+            torch.cuda.synchronize()
+            ms, n = q.qmoe_timing_read("qmv")
+            assert n == 1 and 0.0 < ms < 50.0
+    finally:
+        q.qmoe_timing_enable(None)
