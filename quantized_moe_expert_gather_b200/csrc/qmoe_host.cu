@@ -71,6 +71,30 @@ LaunchTimer::LaunchTimer(const char* kernel, cudaStream_t stream) {
   slot_ = s;
 }
 
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 1;
+  }
+  return cache[dev];
+}
+
+cudaError_t make_tmap_2d_u32(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
+                             int box_inner, int box_rows, bool swizzle128) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, base, inner, rows, box_inner,
+                   box_rows, swizzle128);
+}
+cudaError_t make_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
+                              int box_inner, int box_rows, bool swizzle128) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, rows, box_inner,
+                   box_rows, swizzle128);
+}
+
 }  // namespace qmoe
 
 extern "C" {
