@@ -54,7 +54,8 @@ enum {
   QMOE_ERR_DTYPE = -2,        /* unsupported dtype code                          */
   QMOE_ERR_UNSUPPORTED = -3,  /* bits / group / K combination not supported     */
   QMOE_ERR_WORKSPACE = -4,    /* workspace missing or smaller than required      */
-  QMOE_ERR_CUDA = -5          /* a kernel launch failed                          */
+  QMOE_ERR_CUDA = -5,         /* a kernel launch failed                          */
+  QMOE_ERR_TOO_LARGE = -6     /* beyond the fixed capacity of qmoe_gather_qmm_noalloc */
 };
 
 enum { QMOE_DTYPE_BF16 = 0, QMOE_DTYPE_F32 = 1 };
@@ -163,6 +164,31 @@ QMOE_API int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, i
                     int64_t E, int64_t N, int group, int bits, const uint32_t* lhs_indices,
                     const uint32_t* rhs_indices, int64_t B, int sorted_indices, void* workspace,
                     size_t workspace_bytes, qmoe_bf16* y, int* d_status, qmoe_stream stream);
+
+/*
+ * qmoe_gather_qmm_noalloc -- the same product as qmoe_gather_qmm for callers that
+ * cannot allocate device memory.  The pages have no counterpart: this entry point
+ * exists because some callers can neither call cudaMalloc nor hand the library a
+ * workspace -- e.g. a plugin that is given only its input and output tensors by a
+ * host framework that owns all device memory, or a serving loop that must not call
+ * cudaMalloc (it can synchronise the device) between requests.
+ *   Arguments as qmoe_gather_qmm, without the workspace.  The routing metadata lives
+ *   in a fixed 128 KiB array in device memory inside the library (one copy per GPU
+ *   that loads the library, held until the process exits).  The call allocates
+ *   nothing and runs the streaming kernel path.
+ *   Limits: B*M <= 4096 routed rows and E <= 1024 experts; larger problems return
+ *   QMOE_ERR_TOO_LARGE before any launch.
+ *   The first call on a device looks up the array's device address (with that device
+ *   current); make that first call before any stream capture.
+ *   All calls share the array: calls that overlap on the GPU (other streams, other
+ *   threads) race on it and must be serialised by the caller.
+ */
+QMOE_API int qmoe_gather_qmm_noalloc(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
+                                     const uint32_t* codes, const qmoe_bf16* scales,
+                                     const qmoe_bf16* biases, int64_t E, int64_t N, int group,
+                                     int bits, const uint32_t* lhs_indices,
+                                     const uint32_t* rhs_indices, int64_t B, int sorted_indices,
+                                     qmoe_bf16* y, int* d_status, qmoe_stream stream);
 
 /*
  * qmoe_sort_by_expert -- stable counting sort of routed rows by expert ([P5] Change:

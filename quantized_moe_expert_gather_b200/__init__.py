@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "QmoeError", "load", "library_path", "qmoe_status_string", "qmoe_launch_count", "qmoe_timing_enable", "qmoe_timing_read",
     "qmoe_quantize", "qmoe_dequantize", "qmoe_qmm", "qmoe_gather_qmm",
-    "qmoe_gather_qmm_workspace_size", "qmoe_sort_by_expert", "qmoe_tile_table",
+    "qmoe_gather_qmm_workspace_size", "qmoe_gather_qmm_noalloc", "qmoe_sort_by_expert", "qmoe_tile_table",
     "qmoe_switch_glu", "qmoe_switch_glu_workspace_size", "qmoe_moe_combine", "QWeight",
     "QMOE_DEV_BAD_INDEX", "QMOE_DEV_TIMEOUT", "EXPORTED",
 ]
@@ -56,6 +56,8 @@ _SIGS = {
     "qmoe_gather_qmm_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i64]),
     "qmoe_gather_qmm": (_i32, [_p, _i64, _i64, _i64, _p, _p, _p, _i64, _i64, _i32, _i32,
                                _p, _p, _i64, _i32, _p, _sz, _p, _p, _p]),
+    "qmoe_gather_qmm_noalloc": (_i32, [_p, _i64, _i64, _i64, _p, _p, _p, _i64, _i64, _i32,
+                                       _i32, _p, _p, _i64, _i32, _p, _p, _p]),
     "qmoe_sort_by_expert_workspace_size": (_sz, [_i64, _i64]),
     "qmoe_sort_by_expert": (_i32, [_p, _i64, _i64, _p, _p, _p, _p, _sz, _p, _p]),
     "qmoe_tile_table": (_i32, [_p, _i64, _i32, _p, _i64, _p, _p, _p]),
@@ -228,6 +230,30 @@ def qmoe_gather_qmm(x, codes, scales, biases, lhs_indices=None, rhs_indices=None
         _ptr(x), xb, M, K, _ptr(codes), _ptr(scales), _ptr(biases), E, N, group, bits,
         _ptr(lhs_indices), _ptr(rhs_indices), B, int(bool(sorted_indices)), _ptr(ws), ws.numel(),
         _ptr(y), _ptr(status), _stream()))
+    return y
+
+
+def qmoe_gather_qmm_noalloc(x, codes, scales, biases, lhs_indices=None, rhs_indices=None,
+                            group: int = 64, bits: int = 4, sorted_indices: bool = False,
+                            out=None, status=None):
+    """As :func:`qmoe_gather_qmm`, for callers that cannot allocate device scratch:
+    the library keeps the routing metadata in its own fixed device array (B*M <= 4096,
+    E <= 1024; overlapping calls race on it).  Pass ``out`` to allocate nothing here."""
+    _need(x, "x", _BF16)
+    _need(codes, "codes", _CODES)
+    xb, M, K = x.shape
+    E, N = codes.shape[0], codes.shape[1]
+    if rhs_indices is not None:
+        B = rhs_indices.numel()
+    elif lhs_indices is not None:
+        B = lhs_indices.numel()
+    else:
+        B = max(xb, E)
+    y = out if out is not None else torch.empty((B, M, N), dtype=torch.bfloat16, device=x.device)
+    _check("qmoe_gather_qmm_noalloc", load().qmoe_gather_qmm_noalloc(
+        _ptr(x), xb, M, K, _ptr(codes), _ptr(scales), _ptr(biases), E, N, group, bits,
+        _ptr(lhs_indices), _ptr(rhs_indices), B, int(bool(sorted_indices)), _ptr(y),
+        _ptr(status), _stream()))
     return y
 
 

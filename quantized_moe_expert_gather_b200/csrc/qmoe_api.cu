@@ -122,6 +122,8 @@ const char* qmoe_status_string(int status) {
     case QMOE_ERR_UNSUPPORTED: return "QMOE_ERR_UNSUPPORTED: unsupported bits/group/K combination";
     case QMOE_ERR_WORKSPACE: return "QMOE_ERR_WORKSPACE: workspace missing or too small";
     case QMOE_ERR_CUDA: return "QMOE_ERR_CUDA: kernel launch failed";
+    case QMOE_ERR_TOO_LARGE:
+      return "QMOE_ERR_TOO_LARGE: problem exceeds the fixed scratch capacity (B*M <= 4096, E <= 1024)";
     default: return "unknown qmoe status";
   }
 }
