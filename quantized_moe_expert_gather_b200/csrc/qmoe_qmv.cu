@@ -9,13 +9,15 @@
 // The tile table makes every touched expert's packed weights stream from HBM once
 // per tile (MLX issue #4509: M=1 decode must still reach full bandwidth).
 //
-// Structure (one persistent CTA per SM, 9 warps):
-//   * warp 8 (producer) walks the CTA's contiguous range of (tile, 16-row block)
+// Structure (one persistent CTA per SM, CW consumer warps + 1 producer warp):
+//   * the last warp (producer) walks the CTA's contiguous range of (tile, 16-row block)
 //     units and, per K-chunk, loads the 16 packed rows with 2-D TMA boxes of
 //     128 B x 16 rows (128B-swizzled, so the consumers' row-strided reads are free
 //     of bank conflicts) and the matching scales/biases with cp.async, into a ring
 //     of stages guarded by full/empty mbarriers;
-//   * warps 0..7 (consumers) split each chunk's groups.  A lane turns its packed
+//   * warps 0..CW-1 (consumers) split each chunk's groups.  Each lane prefetches the
+//     activation values its MMA fragments need one chunk ahead into registers (the
+//     loads of chunk c+1 are in flight while chunk c is computed).  A lane turns its packed
 //     codes into bf16 "128 + q" (or "2048 + 16*hi" for the high nibble of 8-bit
 //     codes) with one LOP3 per code pair and feeds mma.sync m16n8k16 with W as the
 //     16-row A operand and up to 8 routed rows as the B operand.  Each MMA k-step
@@ -31,6 +33,7 @@
 #include <cstdio>
 #include <cudaTypedefs.h>
 #include <mutex>
+#include <type_traits>
 
 #include "qmoe_common.cuh"
 #include "qmoe_internal.h"
@@ -39,28 +42,36 @@
 namespace qmoe {
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kRows = 16;             // output channels per unit (MMA M)
 constexpr int kSmemBudget = 225 * 1024;
 
+// Consumer warps: 16 where the register budget allows (more warps hide the shared
+// memory and MMA latencies of the streaming loop), else 8.
+template <int BITS, int GS, int NT>
+constexpr int consumer_warps() {
+  return (BITS == 4 && NT == 1 && GS <= 64) ? 16 : 8;
+}
+
 template <int BITS, int GS, int NMAT, int NT>
 struct Cfg {
+  static constexpr int CW = consumer_warps<BITS, GS, NT>();
+  static constexpr int THREADS = (CW + 1) * 32;
   static constexpr int KB_BYTES = GS * BITS / 8;                 // one group of one row
-  static constexpr int CHUNK_ROW_BYTES = std::max(512, KB_BYTES * kConsumerWarps);
+  static constexpr int CHUNK_ROW_BYTES = std::max(512, KB_BYTES * CW);
   static constexpr int KB_PER_CHUNK = CHUNK_ROW_BYTES / KB_BYTES;
-  static constexpr int KB_PER_WARP = KB_PER_CHUNK / kConsumerWarps;
+  static constexpr int KB_PER_WARP = KB_PER_CHUNK / CW;
   static constexpr int BOXES = CHUNK_ROW_BYTES / 128;
   static constexpr int LANE_BYTES = KB_BYTES / 4;                // per row, per lane
   static constexpr int WORDS = LANE_BYTES / 4;
   static constexpr int CODE_BYTES = NMAT * BOXES * 2048;
   static constexpr int SB_BYTES = NMAT * 2 * kRows * KB_PER_CHUNK * 2;
   static constexpr int STAGE_BYTES = ((CODE_BYTES + SB_BYTES) + 1023) / 1024 * 1024;
-  static constexpr int RED_BYTES = kConsumerWarps * NMAT * NT * kRows * 8 * 4;
+  static constexpr int RED_BYTES = CW * NMAT * NT * kRows * 8 * 4;
   static constexpr int STAGES =
       std::min(8, (kSmemBudget - RED_BYTES - 1024) / STAGE_BYTES);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RED_BYTES + 2 * STAGES * 8 + 64;
   static constexpr uint32_t TMA_BYTES = CODE_BYTES;
+  static_assert((kRows * KB_PER_CHUNK * 2) % 128 == 0, "scale/bias TMA boxes must stay 128-byte aligned");
   static constexpr float OFFSET = BITS == 4 ? 128.0f : 2176.0f;
   static_assert(STAGES >= 3, "too few pipeline stages");
   static_assert(KB_PER_WARP >= 1, "chunk smaller than one group per warp");
@@ -68,6 +79,7 @@ struct Cfg {
 
 struct alignas(64) QmvParams {
   CUtensorMap tmap[2];          // packed codes of each weight stack, [E*N rows, K*bits/32 words]
+  CUtensorMap tmap_sb[2][2];    // [stack][scales|biases], [E*N rows, K/group] bf16
   const uint16_t* scales[2];
   const uint16_t* biases[2];
   const uint16_t* x;
@@ -78,7 +90,8 @@ struct alignas(64) QmvParams {
   const uint32_t* num_tiles;
   int64_t dense_rows;
   int64_t N, K, E;
-  int sb_vec;                   // byte width of the scale/bias copy pieces (2: plain copies)
+  int sb_tma;                   // scales/biases by TMA (row pitch a multiple of 16 bytes)
+  int sb_vec;                   // else: byte width of the copy pieces (2: plain copies)
   int* d_status;
   ProfSlot* prof;
 };
@@ -115,8 +128,10 @@ __device__ __forceinline__ uint32_t swz(int row, int c) {
 }
 
 template <int BITS, int GS, int NMAT, int NT>
-__global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant__ QmvParams p) {
+__global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
+    qmv_kernel(const __grid_constant__ QmvParams p) {
   using C = Cfg<BITS, GS, NMAT, NT>;
+  constexpr int kConsumerWarps = C::CW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -128,7 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1 + 32);                 // producer's expect_tx + 32 cp.async arrivals
+      // producer's expect_tx (+ 32 per-lane arrivals when scales/biases are copied by lanes)
+      mbar_init(&full[s], p.sb_tma ? 1 : 1 + 32);
       mbar_init(&empty[s], kConsumerWarps);
     }
     *abort_flag = 0;
@@ -147,8 +163,14 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      tma_prefetch_desc(&p.tmap[0]);
-      if (NMAT > 1) tma_prefetch_desc(&p.tmap[1]);
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        tma_prefetch_desc(&p.tmap[m]);
+        if (p.sb_tma) {
+          tma_prefetch_desc(&p.tmap_sb[m][0]);
+          tma_prefetch_desc(&p.tmap_sb[m][1]);
+        }
+      }
     }
     uint32_t it = 0;
     bool aborted = false;
@@ -169,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
         }
         uint8_t* st = smem + stage * C::STAGE_BYTES;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], C::TMA_BYTES);
+          mbar_arrive_expect_tx(&full[stage], C::TMA_BYTES + (p.sb_tma ? C::SB_BYTES : 0u));
           const int32_t xw = static_cast<int32_t>(ch * (C::CHUNK_ROW_BYTES / 4));
 #pragma unroll
           for (int m = 0; m < NMAT; ++m)
@@ -177,7 +199,17 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
             for (int bx = 0; bx < C::BOXES; ++bx)
               tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[m], &full[stage], xw + bx * 32,
                           static_cast<int32_t>(row0));
+          if (p.sb_tma) {
+            const int32_t xg = static_cast<int32_t>(ch * C::KB_PER_CHUNK);
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+              for (int arr = 0; arr < 2; ++arr)
+                tma_load_2d(st + C::CODE_BYTES + (m * 2 + arr) * kRows * C::KB_PER_CHUNK * 2,
+                            &p.tmap_sb[m][arr], &full[stage], xg, static_cast<int32_t>(row0));
+          }
         }
+        if (p.sb_tma) continue;
         // scales and biases: [mat][s|b][16 rows][KB_PER_CHUNK] bf16
         const int64_t kb0 = ch * C::KB_PER_CHUNK;
         const int ngroups = static_cast<int>(imin64(C::KB_PER_CHUNK, KB_TOTAL - kb0));
@@ -219,22 +251,62 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
   // ----------------------------------------------------------------- consumers
   const int g = lane >> 2, t = lane & 3;
   const uint32_t ONES = 0x3F803F80u;  // bf16x2 (1, 1)
-  uint32_t it = 0;
-  for (int64_t u = u_begin; u < u_end; ++u) {
-    const TileInfo ti = tile_info<NT>(p, u / NB);
-    const int64_t n0 = (u % NB) * kRows;
-    // x rows of the token slots this lane feeds into the B operand
-    const uint16_t* xrow[NT];
+  // Activation values of one chunk for this lane: [k-block][token set][word]; 16 B per
+  // 4-bit word (8 codes), 8 B per 8-bit word (4 codes).
+  using XV = typename std::conditional<BITS == 4, uint4, uint2>::type;
+  XV xc[C::KB_PER_WARP][NT][C::WORDS], xn[C::KB_PER_WARP][NT][C::WORDS];
+
+  // Row pointers of this lane's token slots for unit u (null for empty slots).
+  auto unit_rows = [&](int64_t u, TileInfo& ti, const uint16_t* (&rows)[NT]) {
+    ti = tile_info<NT>(p, u / NB);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint32_t slot = g + 8 * nt;
-      xrow[nt] = nullptr;
+      rows[nt] = nullptr;
       if (slot < ti.valid) {
         const uint32_t pos = ti.row_start + slot;
         const uint32_t sr = p.src_row ? p.src_row[pos] : pos;
-        xrow[nt] = p.x + static_cast<int64_t>(sr) * p.K;
+        rows[nt] = p.x + static_cast<int64_t>(sr) * p.K;
       }
     }
+  };
+  // Issues the loads of chunk `ch` for the given rows into `dst`.
+  auto load_x = [&](const uint16_t* const (&rows)[NT], int64_t ch, XV (&dst)[C::KB_PER_WARP][NT][C::WORDS]) {
+#pragma unroll
+    for (int i = 0; i < C::KB_PER_WARP; ++i) {
+      const int64_t kb = ch * C::KB_PER_CHUNK + warp + kConsumerWarps * i;
+      const int64_t k0 = kb * GS + t * (GS / 4);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < C::WORDS; ++j) {
+          if constexpr (BITS == 4) {
+            dst[i][nt][j] = make_uint4(0, 0, 0, 0);
+            if (rows[nt] != nullptr && kb < KB_TOTAL) dst[i][nt][j] = ldg_nc_v4(rows[nt] + k0 + 8 * j);
+          } else {
+            dst[i][nt][j] = make_uint2(0, 0);
+            if (rows[nt] != nullptr && kb < KB_TOTAL) dst[i][nt][j] = ldg_nc_v2(rows[nt] + k0 + 4 * j);
+          }
+        }
+    }
+  };
+
+  uint32_t it = 0;
+  TileInfo ti_next{};
+  const uint16_t* rows_next[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) rows_next[nt] = nullptr;
+  if (u_begin < u_end) {
+    unit_rows(u_begin, ti_next, rows_next);
+    load_x(rows_next, 0, xn);
+  }
+  for (int64_t u = u_begin; u < u_end; ++u) {
+    const TileInfo ti = ti_next;
+    const uint16_t* rows[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) rows[nt] = rows_next[nt];
+    const int64_t n0 = (u % NB) * kRows;
+    if (u + 1 < u_end) unit_rows(u + 1, ti_next, rows_next);  // one unit ahead
     float acc[NMAT][NT][4];
 #pragma unroll
     for (int m = 0; m < NMAT; ++m)
@@ -244,6 +316,17 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
         for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.f;
 
     for (int64_t ch = 0; ch < NCH; ++ch, ++it) {
+      // take this chunk's activations; start the next chunk's loads
+#pragma unroll
+      for (int i = 0; i < C::KB_PER_WARP; ++i)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int j = 0; j < C::WORDS; ++j) xc[i][nt][j] = xn[i][nt][j];
+      if (ch + 1 < NCH)
+        load_x(rows, ch + 1, xn);
+      else if (u + 1 < u_end)
+        load_x(rows_next, 0, xn);
       const int stage = it % C::STAGES;
       bool ok = false;
       if (!*abort_flag) {
@@ -258,7 +341,6 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
           const int ikb = warp + kConsumerWarps * i;
           const int64_t kb = ch * C::KB_PER_CHUNK + ikb;
           if (kb >= KB_TOTAL) break;
-          const int64_t k0 = kb * GS + t * (GS / 4);  // first k of this lane's codes
           // ---- B operand: x values of this lane's codes, permuted to the MMA k order
           uint32_t bfr[NT][C::WORDS][2][2];
 #pragma unroll
@@ -266,15 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
 #pragma unroll
             for (int j = 0; j < C::WORDS; ++j) {
               if constexpr (BITS == 4) {
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (xrow[nt]) v = ldg_nc_v4(xrow[nt] + k0 + 8 * j);
+                const uint4 v = xc[i][nt][j];
                 bfr[nt][j][0][0] = prmt(v.x, v.z, 0x5410);
                 bfr[nt][j][0][1] = prmt(v.x, v.z, 0x7632);
                 bfr[nt][j][1][0] = prmt(v.y, v.w, 0x5410);
                 bfr[nt][j][1][1] = prmt(v.y, v.w, 0x7632);
               } else {
-                uint2 v = make_uint2(0, 0);
-                if (xrow[nt]) v = ldg_nc_v2(xrow[nt] + k0 + 4 * j);
+                const uint2 v = xc[i][nt][j];
                 bfr[nt][j][0][0] = prmt(v.x, v.y, 0x5410);
                 bfr[nt][j][0][1] = prmt(v.x, v.y, 0x7632);
                 bfr[nt][j][1][0] = bfr[nt][j][0][0];
@@ -413,8 +493,20 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const __grid_constant_
 }
 
 template <int BITS, int GS, int NMAT, int NT>
-cudaError_t launch_cfg(QmvParams prm, cudaStream_t stream) {
+cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
   using C = Cfg<BITS, GS, NMAT, NT>;
+  const int64_t gpr = a.K / GS;
+  prm.sb_tma = (gpr % 8 == 0) ? 1 : 0;
+  if (prm.sb_tma) {
+    for (int m = 0; m < a.nmat; ++m) {
+      const uint16_t* arrs[2] = {a.w[m].scales, a.w[m].biases};
+      for (int arr = 0; arr < 2; ++arr) {
+        cudaError_t e = make_tmap_2d_bf16(&prm.tmap_sb[m][arr], arrs[arr], gpr, a.E * a.N,
+                                          C::KB_PER_CHUNK, kRows, /*swizzle128=*/false);
+        if (e != cudaSuccess) return e;
+      }
+    }
+  }
   auto kern = qmv_kernel<BITS, GS, NMAT, NT>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -425,17 +517,19 @@ cudaError_t launch_cfg(QmvParams prm, cudaStream_t stream) {
   if (attr_err != cudaSuccess) return attr_err;
   LaunchTimer timer(NMAT == 2 ? "qmv_glu" : "qmv", stream);
   prm.prof = timer.slot();
-  kern<<<sm_count(), kThreads, C::SMEM_BYTES + 1024, stream>>>(prm);
+  kern<<<sm_count(), C::THREADS, C::SMEM_BYTES + 1024, stream>>>(prm);
   count_launch();
   return cudaGetLastError();
 }
 
 template <int BITS, int GS>
-cudaError_t launch_bits_gs(const QmvParams& prm, int nmat, int nt, cudaStream_t stream) {
-  if (nmat == 2) {
-    return nt == 2 ? launch_cfg<BITS, GS, 2, 2>(prm, stream) : launch_cfg<BITS, GS, 2, 1>(prm, stream);
+cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cudaStream_t stream) {
+  if (a.nmat == 2) {
+    return nt == 2 ? launch_cfg<BITS, GS, 2, 2>(prm, a, stream)
+                   : launch_cfg<BITS, GS, 2, 1>(prm, a, stream);
   }
-  return nt == 2 ? launch_cfg<BITS, GS, 1, 2>(prm, stream) : launch_cfg<BITS, GS, 1, 1>(prm, stream);
+  return nt == 2 ? launch_cfg<BITS, GS, 1, 2>(prm, a, stream)
+                 : launch_cfg<BITS, GS, 1, 1>(prm, a, stream);
 }
 
 }  // namespace
@@ -465,13 +559,13 @@ cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
   prm.d_status = a.d_status;
   const int nt = a.bm > 8 ? 2 : 1;
   if (a.bits == 4) {
-    if (a.group == 32) return launch_bits_gs<4, 32>(prm, a.nmat, nt, stream);
-    if (a.group == 64) return launch_bits_gs<4, 64>(prm, a.nmat, nt, stream);
-    return launch_bits_gs<4, 128>(prm, a.nmat, nt, stream);
+    if (a.group == 32) return launch_bits_gs<4, 32>(prm, a, nt, stream);
+    if (a.group == 64) return launch_bits_gs<4, 64>(prm, a, nt, stream);
+    return launch_bits_gs<4, 128>(prm, a, nt, stream);
   }
-  if (a.group == 32) return launch_bits_gs<8, 32>(prm, a.nmat, nt, stream);
-  if (a.group == 64) return launch_bits_gs<8, 64>(prm, a.nmat, nt, stream);
-  return launch_bits_gs<8, 128>(prm, a.nmat, nt, stream);
+  if (a.group == 32) return launch_bits_gs<8, 32>(prm, a, nt, stream);
+  if (a.group == 64) return launch_bits_gs<8, 64>(prm, a, nt, stream);
+  return launch_bits_gs<8, 128>(prm, a, nt, stream);
 }
 
 }  // namespace qmoe
