@@ -66,7 +66,9 @@ struct Cfg {
   static constexpr int CODE_BYTES = NMAT * BOXES * 2048;
   static constexpr int SB_BYTES = NMAT * 2 * kRows * KB_PER_CHUNK * 2;
   static constexpr int STAGE_BYTES = ((CODE_BYTES + SB_BYTES) + 1023) / 1024 * 1024;
-  static constexpr int RED_BYTES = CW * NMAT * NT * kRows * 8 * 4;
+  // per-warp partial sums, double-buffered: [2][CW][NMAT][NT][16 rows][8 tokens] fp32
+  static constexpr int RED_SLICE = CW * NMAT * NT * kRows * 8;
+  static constexpr int RED_BYTES = 2 * RED_SLICE * 4;
   static constexpr int STAGES =
       std::min(8, (kSmemBudget - RED_BYTES - 1024) / STAGE_BYTES);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RED_BYTES + 2 * STAGES * 8 + 64;
@@ -90,6 +92,7 @@ struct alignas(64) QmvParams {
   const uint32_t* num_tiles;
   int64_t dense_rows;
   int64_t N, K, E;
+  int pair;                     // 1: one weight stack, a unit is two adjacent 16-row blocks
   int sb_tma;                   // scales/biases by TMA (row pitch a multiple of 16 bytes)
   int sb_vec;                   // else: byte width of the copy pieces (2: plain copies)
   int* d_status;
@@ -155,7 +158,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 
   const int64_t KB_TOTAL = p.K / GS;
   const int64_t NCH = (KB_TOTAL + C::KB_PER_CHUNK - 1) / C::KB_PER_CHUNK;
-  const int64_t NB = (p.N + kRows - 1) / kRows;
+  const int unit_rows = p.pair ? 2 * kRows : kRows;  // output channels per unit
+  const int64_t NB = (p.N + unit_rows - 1) / unit_rows;
   const int64_t units = num_tiles<NT>(p) * NB;
   const int64_t u_begin = units * blockIdx.x / gridDim.x;
   const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
@@ -176,9 +180,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
     bool aborted = false;
     for (int64_t u = u_begin; u < u_end && !aborted; ++u) {
       const TileInfo ti = tile_info<NT>(p, u / NB);
-      const int64_t n0 = (u % NB) * kRows;
+      const int64_t n0 = (u % NB) * unit_rows;
       const int64_t row0 = static_cast<int64_t>(ti.expert) * p.N + n0;
-      const int nrows = static_cast<int>(imin64(kRows, p.N - n0));
       for (int64_t ch = 0; ch < NCH; ++ch, ++it) {
         const int stage = it % C::STAGES;
         const uint32_t round = it / C::STAGES;
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 #pragma unroll
             for (int bx = 0; bx < C::BOXES; ++bx)
               tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[m], &full[stage], xw + bx * 32,
-                          static_cast<int32_t>(row0));
+                          static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
           if (p.sb_tma) {
             const int32_t xg = static_cast<int32_t>(ch * C::KB_PER_CHUNK);
 #pragma unroll
@@ -206,7 +209,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 #pragma unroll
               for (int arr = 0; arr < 2; ++arr)
                 tma_load_2d(st + C::CODE_BYTES + (m * 2 + arr) * kRows * C::KB_PER_CHUNK * 2,
-                            &p.tmap_sb[m][arr], &full[stage], xg, static_cast<int32_t>(row0));
+                            &p.tmap_sb[m][arr], &full[stage], xg,
+                            static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
           }
         }
         if (p.sb_tma) continue;
@@ -214,14 +218,18 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
         const int64_t kb0 = ch * C::KB_PER_CHUNK;
         const int ngroups = static_cast<int>(imin64(C::KB_PER_CHUNK, KB_TOTAL - kb0));
         const int pieces = ngroups * 2 / p.sb_vec;
-        const int tasks = NMAT * 2 * nrows * pieces;
+        // rows of each 16-row block inside [0, N): the tail block of a pair may be short
+        const int nrows = static_cast<int>(imin64(kRows, p.N - n0));
+        const int tasks = NMAT * 2 * kRows * pieces;
         uint16_t* sb = reinterpret_cast<uint16_t*>(st + C::CODE_BYTES);
         for (int tk = lane; tk < tasks; tk += 32) {
           const int piece = tk % pieces;
-          const int rr = (tk / pieces) % nrows;
-          const int arr = (tk / (pieces * nrows)) % 2;
-          const int m = tk / (pieces * nrows * 2);
-          const uint16_t* src = (arr ? p.biases[m] : p.scales[m]) + (row0 + rr) * KB_TOTAL + kb0;
+          const int rr = (tk / pieces) % kRows;
+          const int arr = (tk / (pieces * kRows)) % 2;
+          const int m = tk / (pieces * kRows * 2);
+          const int mrow = p.pair ? kRows * m + rr : rr;  // row inside the unit
+          if (mrow >= (p.pair ? static_cast<int>(imin64(2 * kRows, p.N - n0)) : nrows)) continue;
+          const uint16_t* src = (arr ? p.biases[m] : p.scales[m]) + (row0 + mrow) * KB_TOTAL + kb0;
           uint16_t* dst = sb + ((m * 2 + arr) * kRows + rr) * C::KB_PER_CHUNK;
           const int off = piece * (p.sb_vec / 2);
           if (p.sb_vec == 16)
@@ -257,7 +265,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
   XV xc[C::KB_PER_WARP][NT][C::WORDS], xn[C::KB_PER_WARP][NT][C::WORDS];
 
   // Row pointers of this lane's token slots for unit u (null for empty slots).
-  auto unit_rows = [&](int64_t u, TileInfo& ti, const uint16_t* (&rows)[NT]) {
+  auto tile_rows = [&](int64_t u, TileInfo& ti, const uint16_t* (&rows)[NT]) {
     ti = tile_info<NT>(p, u / NB);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -297,7 +305,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) rows_next[nt] = nullptr;
   if (u_begin < u_end) {
-    unit_rows(u_begin, ti_next, rows_next);
+    tile_rows(u_begin, ti_next, rows_next);
     load_x(rows_next, 0, xn);
   }
   for (int64_t u = u_begin; u < u_end; ++u) {
@@ -305,8 +313,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
     const uint16_t* rows[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) rows[nt] = rows_next[nt];
-    const int64_t n0 = (u % NB) * kRows;
-    if (u + 1 < u_end) unit_rows(u + 1, ti_next, rows_next);  // one unit ahead
+    const int64_t n0 = (u % NB) * unit_rows;
+    if (u + 1 < u_end) tile_rows(u + 1, ti_next, rows_next);  // one unit ahead
     float acc[NMAT][NT][4];
 #pragma unroll
     for (int m = 0; m < NMAT; ++m)
@@ -451,43 +459,61 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
       if (lane == 0) mbar_arrive(&empty[stage]);
     }
 
-    // ---- cross-warp reduction and epilogue
+    // ---- cross-warp reduction: each warp stores its partial sums (valid token
+    // columns only) in its own slot; the epilogue adds the slots in warp order, so the
+    // result does not depend on timing.  Two buffers alternate between units: one
+    // barrier per unit suffices.
+    float* ub = red + ((u - u_begin) & 1) * C::RED_SLICE;
+    if (!*abort_flag) {
 #pragma unroll
-    for (int m = 0; m < NMAT; ++m)
+      for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float* r = red + (((warp * NMAT + m) * NT + nt) * kRows) * 8;
-        r[g * 8 + 2 * t] = acc[m][nt][0];
-        r[g * 8 + 2 * t + 1] = acc[m][nt][1];
-        r[(g + 8) * 8 + 2 * t] = acc[m][nt][2];
-        r[(g + 8) * 8 + 2 * t + 1] = acc[m][nt][3];
-      }
+        for (int nt = 0; nt < NT; ++nt) {
+          float* r = ub + (((warp * NMAT + m) * NT + nt) * kRows) * 8;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (static_cast<uint32_t>(nt * 8 + 2 * t + j) < ti.valid) {
+              r[g * 8 + 2 * t + j] = acc[m][nt][j];
+              r[(g + 8) * 8 + 2 * t + j] = acc[m][nt][2 + j];
+            }
+          }
+        }
+    }
     named_bar_sync(1, kConsumerWarps * 32);
+    // ---- epilogue: one thread per (row, token) entry
     const int tid = threadIdx.x;
-    if (tid < NT * 128 && !*abort_flag) {
+    if (tid < NT * 128) {
       const int nt = tid / 128, rem = tid % 128, tok = rem / 16, row = rem % 16;
       const uint32_t slot = nt * 8 + tok;
-      if (slot < ti.valid && n0 + row < p.N) {
+      if (!*abort_flag && slot < ti.valid) {
         float v[NMAT];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-          float s = 0.f;
+          float sum = 0.f;
 #pragma unroll
           for (int w = 0; w < kConsumerWarps; ++w)
-            s += red[(((w * NMAT + m) * NT + nt) * kRows + row) * 8 + tok];
-          v[m] = s;
-        }
-        float out = v[0];
-        if constexpr (NMAT == 2) {
-          const float gte = v[1];
-          out = v[0] * (gte / (1.0f + expf(-gte)));
+            sum += ub[(((w * NMAT + m) * NT + nt) * kRows + row) * 8 + tok];
+          v[m] = sum;
         }
         const uint32_t pos = ti.row_start + slot;
         const uint32_t dr = p.dst_row ? p.dst_row[pos] : pos;
-        p.y[static_cast<int64_t>(dr) * p.N + n0 + row] = f32_to_bf16(out);
+        uint16_t* yrow = p.y + static_cast<int64_t>(dr) * p.N;
+        if (p.pair) {
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            const int64_t n = n0 + kRows * m + row;
+            if (n < p.N) yrow[n] = f32_to_bf16(v[m]);
+          }
+        } else if (n0 + row < p.N) {
+          float out = v[0];
+          if constexpr (NMAT == 2) {
+            const float gte = v[1];
+            out = v[0] * (gte / (1.0f + expf(-gte)));
+          }
+          yrow[n0 + row] = f32_to_bf16(out);
+        }
       }
     }
-    named_bar_sync(1, kConsumerWarps * 32);
   }
   if (threadIdx.x == 0) prof_end(p.prof);
 }
@@ -498,8 +524,9 @@ cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
   const int64_t gpr = a.K / GS;
   prm.sb_tma = (gpr % 8 == 0) ? 1 : 0;
   if (prm.sb_tma) {
-    for (int m = 0; m < a.nmat; ++m) {
-      const uint16_t* arrs[2] = {a.w[m].scales, a.w[m].biases};
+    for (int m = 0; m < 2; ++m) {
+      const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
+      const uint16_t* arrs[2] = {wm.scales, wm.biases};
       for (int arr = 0; arr < 2; ++arr) {
         cudaError_t e = make_tmap_2d_bf16(&prm.tmap_sb[m][arr], arrs[arr], gpr, a.E * a.N,
                                           C::KB_PER_CHUNK, kRows, /*swizzle128=*/false);
@@ -515,7 +542,7 @@ cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
                                     C::SMEM_BYTES + 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  LaunchTimer timer(NMAT == 2 ? "qmv_glu" : "qmv", stream);
+  LaunchTimer timer(prm.pair ? "qmv" : "qmv_glu", stream);
   prm.prof = timer.slot();
   kern<<<sm_count(), C::THREADS, C::SMEM_BYTES + 1024, stream>>>(prm);
   count_launch();
@@ -524,12 +551,9 @@ cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
 
 template <int BITS, int GS>
 cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cudaStream_t stream) {
-  if (a.nmat == 2) {
-    return nt == 2 ? launch_cfg<BITS, GS, 2, 2>(prm, a, stream)
-                   : launch_cfg<BITS, GS, 2, 1>(prm, a, stream);
-  }
-  return nt == 2 ? launch_cfg<BITS, GS, 1, 2>(prm, a, stream)
-                 : launch_cfg<BITS, GS, 1, 1>(prm, a, stream);
+  // a single weight stack runs as two adjacent 16-row blocks of that stack
+  return nt == 2 ? launch_cfg<BITS, GS, 2, 2>(prm, a, stream)
+                 : launch_cfg<BITS, GS, 2, 1>(prm, a, stream);
 }
 
 }  // namespace
@@ -537,12 +561,14 @@ cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cuda
 cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
   QmvParams prm{};
   const int64_t words = a.K * a.bits / 32;
-  for (int m = 0; m < a.nmat; ++m) {
-    cudaError_t e = make_tmap_2d_u32(&prm.tmap[m], a.w[m].codes, words, a.E * a.N, 32, 16,
+  prm.pair = a.nmat == 2 ? 0 : 1;
+  for (int m = 0; m < 2; ++m) {
+    const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
+    cudaError_t e = make_tmap_2d_u32(&prm.tmap[m], wm.codes, words, a.E * a.N, 32, 16,
                                      /*swizzle128=*/true);
     if (e != cudaSuccess) return e;
-    prm.scales[m] = a.w[m].scales;
-    prm.biases[m] = a.w[m].biases;
+    prm.scales[m] = wm.scales;
+    prm.biases[m] = wm.biases;
   }
   prm.x = a.x;
   prm.src_row = a.src_row;
