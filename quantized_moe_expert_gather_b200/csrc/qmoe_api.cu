@@ -173,6 +173,7 @@ int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, const qmoe_bf
   a.group = group;
   a.bits = bits;
   a.x = x;
+  a.x_rows = M;
   a.y = y;
   a.dense_rows = M;
   a.d_status = d_status;
@@ -221,6 +222,7 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   a.group = group;
   a.bits = bits;
   a.y = y;
+  a.x_rows = R;  // the tensor-core path reads the expert-ordered copy of x
   a.dst_row = rb.order;
   a.tiles = rb.tiles;
   a.num_tiles = rb.num_tiles;
@@ -346,6 +348,7 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   ug.group = up->group;
   ug.bits = up->bits;
   ug.y = h;
+  ug.x_rows = R;
   ug.tiles = rb.tiles;
   ug.num_tiles = rb.num_tiles;
   ug.d_status = d_status;
@@ -358,6 +361,7 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   dn.group = down->group;
   dn.bits = down->bits;
   dn.x = h;
+  dn.x_rows = R;
   dn.y = y;
   dn.dst_row = mode == 0 ? rb.order : nullptr;
   dn.tiles = rb.tiles;

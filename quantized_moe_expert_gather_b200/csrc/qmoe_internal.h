@@ -87,6 +87,7 @@ struct GemmArgs {
   int64_t E = 1, N = 0, K = 0;
   int group = 64, bits = 4;
   const uint16_t* x = nullptr;       // activation rows, K wide
+  int64_t x_rows = 0;                // rows of x (bound of the activation tensor map)
   const uint32_t* src_row = nullptr; // sorted position -> x row (null: identity)
   uint16_t* y = nullptr;             // output rows, N wide
   const uint32_t* dst_row = nullptr; // sorted position -> y row (null: identity)

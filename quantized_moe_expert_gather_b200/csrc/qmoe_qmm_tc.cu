@@ -1,10 +1,538 @@
-// Tensor-core (tcgen05 / TMEM) gathered quantised matmul for many rows per expert.
+// Tensor-core gathered quantised matmul for many rows per expert (prefill).
+//
+// MLX PR #4567 "[Metal] Gather mm improvement", Proposed changes: rows are sorted by
+// expert and cut into expert-aligned tiles (row start, expert, valid rows), so every
+// tile runs one K loop against one expert's weights.  Each tile of 128 expert-sorted
+// activation rows is multiplied by dequantize(W[e])^T (nuvec-core 0.4.0
+// tests/quantized.rs, gather_qmm_selects_batches) on the 5th-generation tensor cores;
+// with two weight stacks the SwitchGLU epilogue h = silu(gate) * up is fused (MLX
+// issue #4509 repro script, `moe`).
+//
+// One persistent CTA per SM walks a contiguous range of units (tile, block of output
+// channels).  A unit owns two 128x128 fp32 accumulators in tensor memory: (up, gate)
+// for the SwitchGLU, or two adjacent 128-channel blocks of one weight stack.  Warps:
+//   0-3   epilogue: tcgen05.ld of the finished accumulators (one TMEM lane = one row),
+//         silu*mul, bf16 stores to the routed rows;
+//   4     producer: 2-D TMA of the activation tile (128 rows x 64 k, 128B-swizzled),
+//         the packed code tiles (128 rows x 64 codes per stack) and, every 8 groups,
+//         the scales and biases;
+//   5     MMA issuer: owns 512 TMEM columns (two double-buffered unit accumulators),
+//         one thread issues tcgen05.mma kind::f16 (M=128, N=128, K=16) and commits to
+//         mbarriers;
+//   6-13  dequant: one thread per (stack, row) turns 64 packed codes into bf16
+//         q*scale + bias (one rounding) and writes them in the 128B-swizzled K-major
+//         layout the MMA descriptors read.
+// Every mbarrier wait is bounded; a timeout sets QMOE_DEV_TIMEOUT, stops all roles,
+// drains the copies and MMAs in flight and frees the tensor memory.
+#include <algorithm>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "qmoe_common.cuh"
 #include "qmoe_internal.h"
+#include "qmoe_tma.h"
 
 namespace qmoe {
+namespace {
 
-bool qmm_tc_supported(const GemmArgs&) { return false; }
+constexpr int kBM = 128;            // rows per tile = TMEM lanes
+constexpr int kBN = 128;            // output channels per accumulator
+constexpr int kBK = 64;             // k per stage: one 128-byte swizzle atom of bf16
+constexpr int kS1 = 4;              // activation + packed-code ring
+constexpr int kS2 = 2;              // dequantised-weight ring
+constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps = 8;
+constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;  // 448
+constexpr int kTmemCols = 512;      // 2 buffers x 2 accumulators x 128 columns
+constexpr int kSbGroups = 8;        // groups per scale/bias TMA box (16 bytes of bf16)
 
-cudaError_t launch_qmm_tc(const GemmArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+template <int BITS>
+struct TcCfg {
+  static constexpr int A_BYTES = kBM * kBK * 2;                  // 16 KB
+  static constexpr int P_ROW = kBK * BITS / 8;                   // packed bytes per row per stage
+  static constexpr int P_BYTES = 2 * kBM * P_ROW;                // two stacks
+  static constexpr int B_BYTES = 2 * kBN * kBK * 2;              // two stacks, bf16
+  static constexpr int SB_BYTES = 2 * 2 * kBM * kSbGroups * 2;   // [stack][s|b][row][8]
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_P = OFF_A + kS1 * A_BYTES;
+  static constexpr int OFF_B = OFF_P + kS1 * P_BYTES;
+  static constexpr int OFF_SB = OFF_B + kS2 * B_BYTES;
+  static constexpr int OFF_BAR = OFF_SB + 2 * SB_BYTES;
+  static constexpr int SMEM = OFF_BAR + 256;
+  static_assert(OFF_P % 1024 == 0 && OFF_B % 1024 == 0 && OFF_SB % 1024 == 0, "alignment");
+};
+
+struct alignas(64) TcParams {
+  CUtensorMap tm_a;        // activation rows [x_rows, K] bf16, box {64, 128}, 128B swizzle
+  CUtensorMap tm_w[2];     // packed codes [E*N, K*bits/32] u32, box {64*bits/32, 128}
+  CUtensorMap tm_sb[2][2]; // scales / biases [E*N, K/group] bf16, box {8, 128}
+  uint16_t* y;
+  const uint32_t* dst_row;
+  const uint32_t* tiles;
+  const uint32_t* num_tiles;
+  int64_t dense_rows;
+  int64_t N, K;
+  int pair;                // 1: one stack, the two accumulators are adjacent channel blocks
+  int* d_status;
+  ProfSlot* prof;
+};
+
+struct Tile {
+  uint32_t row_start, expert, valid;
+};
+
+__device__ __forceinline__ Tile tc_tile(const TcParams& p, int64_t j) {
+  Tile t;
+  if (p.dense_rows > 0) {
+    t.row_start = static_cast<uint32_t>(j * kBM);
+    t.expert = 0;
+    t.valid = static_cast<uint32_t>(imin64(kBM, p.dense_rows - j * kBM));
+  } else {
+    t.row_start = p.tiles[3 * j];
+    t.expert = p.tiles[3 * j + 1];
+    t.valid = min(p.tiles[3 * j + 2], static_cast<uint32_t>(kBM));
+  }
+  return t;
+}
+
+// ------------------------------------------------------------- tcgen05 helpers
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulation.
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor of a K-major, 128B-swizzled bf16 tile whose rows are
+// 128 bytes (64 k) and whose 8-row groups are 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(const void* smem_tile) {
+  const uint64_t start = (smem_u32(smem_tile) >> 4) & 0x3FFFu;
+  return start | (uint64_t(1) << 16) /* leading offset (unused when swizzled) */ |
+         (uint64_t(1024 >> 4) << 32) /* stride between 8-row groups */ |
+         (uint64_t(1) << 46) /* descriptor version */ | (uint64_t(2) << 61) /* 128B swizzle */;
+}
+
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, M=128, N=128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
+                            (uint32_t(kBM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t bf16x2_of(float lo, float hi) { return pack_bf16x2(lo, hi); }
+
+// 8 packed 4-bit codes (one word, k ascending) -> 8 bf16 of q*s + b (one rounding each).
+__device__ __forceinline__ uint4 dequant_word4(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
+  const uint32_t ws = w >> 4;
+  const __nv_bfloat162 off = __floats2bfloat162_rn(128.f, 128.f);
+  uint32_t out[4];
+#pragma unroll
+  for (int pp = 0; pp < 4; ++pp) {
+    // byte pp of w (low nibble: code 2pp) -> bits 0..3; byte pp of w>>4 (code 2pp+1) -> 16..19
+    const uint32_t sel = pp | (pp << 4) | ((4 + pp) << 8) | ((4 + pp) << 12);
+    const uint32_t y = and_or(prmt(w, ws, sel), 0x000F000Fu, 0x43004300u);  // 128 + q
+    __nv_bfloat162 q2 = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&y), off);  // exact
+    __nv_bfloat162 v = __hfma2(q2, s2, b2);
+    out[pp] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// 4 packed 8-bit codes -> 4 bf16 of q*s + b (fp32 fma, then one rounding to bf16).
+__device__ __forceinline__ uint2 dequant_word8(uint32_t w, float s, float b) {
+  float v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t f = prmt(w, 0x4B000000u, k | (4 << 4) | (4 << 8) | (7 << 12));  // 2^23 + q
+    const float q = __uint_as_float(f) - 8388608.0f;
+    v[k] = fmaf(q, s, b);
+  }
+  return make_uint2(bf16x2_of(v[0], v[1]), bf16x2_of(v[2], v[3]));
+}
+
+template <int BITS, int GS>
+__global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_constant__ TcParams p) {
+  using C = TcCfg<BITS>;
+  // stages covered by one scale/bias box of kSbGroups groups
+  constexpr int KS_SB = kSbGroups * GS / kBK;
+  static_assert(KS_SB >= 1 && (kSbGroups * GS) % kBK == 0, "group size");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full1 = bars;                 // [kS1] TMA tx (activation + packed)
+  uint64_t* empty1 = full1 + kS1;         // [kS1] MMA commit + dequant warps
+  uint64_t* full2 = empty1 + kS1;         // [kS2] dequant warps
+  uint64_t* empty2 = full2 + kS2;         // [kS2] MMA commit
+  uint64_t* full_sb = empty2 + kS2;       // [2] TMA tx
+  uint64_t* empty_sb = full_sb + 2;       // [2] dequant warps
+  uint64_t* tfull = empty_sb + 2;         // [2] MMA commit: accumulator ready
+  uint64_t* tempty = tfull + 2;           // [2] epilogue warps: accumulator drained
+  uint64_t* drain = tempty + 2;           // [1] final MMA commit on the abort path
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kS1; ++s) {
+      mbar_init(&full1[s], 1);
+      mbar_init(&empty1[s], 1 + kDqWarps);
+    }
+    for (int s = 0; s < kS2; ++s) {
+      mbar_init(&full2[s], kDqWarps);
+      mbar_init(&empty2[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full_sb[s], 1);
+      mbar_init(&empty_sb[s], kDqWarps);
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prof_start(p.prof);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_sh;
+
+  const int64_t KS = p.K / kBK;  // k stages per unit
+  const int unit_n = p.pair ? 2 * kBN : kBN;
+  const int64_t NBLK = (p.N + unit_n - 1) / unit_n;
+  const int64_t ntiles = p.dense_rows > 0 ? (p.dense_rows + kBM - 1) / kBM : *p.num_tiles;
+  const int64_t units = ntiles * NBLK;
+  const int64_t u_begin = units * blockIdx.x / gridDim.x;
+  const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == kProdWarp) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_a);
+      uint32_t it = 0, sbit = 0;
+      bool ab = false;
+      for (int64_t u = u_begin; u < u_end && !ab; ++u) {
+        const Tile tl = tc_tile(p, u / NBLK);
+        const int64_t n0 = (u % NBLK) * unit_n;
+        const int64_t wrow = static_cast<int64_t>(tl.expert) * p.N + n0;
+        for (int64_t ks = 0; ks < KS; ++ks) {
+          if (*abort_flag) { ab = true; break; }
+          if (ks % KS_SB == 0) {
+            const uint32_t e = sbit & 1;
+            if (!mbar_wait(&empty_sb[e], ((sbit >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+            mbar_arrive_expect_tx(&full_sb[e], C::SB_BYTES);
+            const int32_t gx = static_cast<int32_t>(ks * kBK / GS);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+              for (int arr = 0; arr < 2; ++arr)
+                tma_load_2d(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
+                            &p.tm_sb[m][arr], &full_sb[e], gx,
+                            static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
+            ++sbit;
+          }
+          const uint32_t s1 = it % kS1;
+          if (!mbar_wait(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+          mbar_arrive_expect_tx(&full1[s1], C::A_BYTES + C::P_BYTES);
+          tma_load_2d(smem + C::OFF_A + s1 * C::A_BYTES, &p.tm_a, &full1[s1],
+                      static_cast<int32_t>(ks * kBK), static_cast<int32_t>(tl.row_start));
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+            tma_load_2d(smem + C::OFF_P + s1 * C::P_BYTES + m * kBM * C::P_ROW, &p.tm_w[m],
+                        &full1[s1], static_cast<int32_t>(ks * kBK * BITS / 32),
+                        static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
+          ++it;
+        }
+      }
+      if (ab) {
+        // let the copies already issued land before the CTA can exit
+        const uint32_t first = it > static_cast<uint32_t>(kS1) ? it - kS1 : 0u;
+        for (uint32_t k = first; k < it; ++k) mbar_wait(&full1[k % kS1], (k / kS1) & 1, nullptr);
+        const uint32_t sfirst = sbit > 2u ? sbit - 2 : 0u;
+        for (uint32_t k = sfirst; k < sbit; ++k) mbar_wait(&full_sb[k & 1], (k >> 1) & 1, nullptr);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tc = 0;
+      bool issued = false;
+      for (int64_t u = u_begin; u < u_end; ++u, ++tc) {
+        if (*abort_flag) break;
+        const uint32_t buf = tc & 1;
+        if (!mbar_wait(&tempty[buf], ((tc >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * (2 * kBN);
+        bool ok = true;
+        for (int64_t ks = 0; ks < KS; ++ks, ++it) {
+          const uint32_t s1 = it % kS1, s2 = it % kS2;
+          if (!mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) ||
+              !mbar_wait(&full2[s2], (it / kS2) & 1, p.d_status)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* a_t = smem + C::OFF_A + s1 * C::A_BYTES;
+          const uint8_t* b_t = smem + C::OFF_B + s2 * C::B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t adesc = sw128_desc(a_t) + 2 * kk;  // +32 bytes along k
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+              const uint64_t bdesc = sw128_desc(b_t + m * kBN * kBK * 2) + 2 * kk;
+              tc_mma(d0 + m * kBN, adesc, bdesc, kIdesc, (ks | kk) != 0 ? 1u : 0u);
+            }
+          }
+          issued = true;
+          tc_commit(&empty1[s1]);
+          tc_commit(&empty2[s2]);
+        }
+        if (!ok) break;
+        tc_commit(&tfull[buf]);
+      }
+      if (*abort_flag && issued) {
+        tc_commit(drain);  // completes when every MMA issued so far has finished
+        mbar_wait(drain, 0, nullptr);
+      }
+    }
+  } else if (warp >= kDqWarp0) {
+    // ------------------------------------------------------------------- dequant
+    const int dq = threadIdx.x - kDqWarp0 * 32;  // 0..255
+    const int m = dq / kBM, row = dq % kBM;
+    uint32_t it = 0, sbit = 0;
+    for (int64_t u = u_begin; u < u_end; ++u) {
+      for (int64_t ks = 0; ks < KS; ++ks, ++it) {
+        if (*abort_flag) break;
+        const uint32_t e = sbit & 1;
+        if (ks % KS_SB == 0 &&
+            !mbar_wait(&full_sb[e], (sbit >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
+        const uint32_t s1 = it % kS1, s2 = it % kS2;
+        if (!mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) ||
+            !mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+        const uint16_t* sbp = reinterpret_cast<const uint16_t*>(smem + C::OFF_SB + e * C::SB_BYTES) +
+                              ((m * 2) * kBM + row) * kSbGroups;
+        const uint16_t* bbp = sbp + kBM * kSbGroups;
+        const int gin = static_cast<int>((ks * kBK / GS) % kSbGroups);
+        const uint8_t* prow = smem + C::OFF_P + s1 * C::P_BYTES + (m * kBM + row) * C::P_ROW;
+        uint8_t* brow = smem + C::OFF_B + s2 * C::B_BYTES + (m * kBN + row) * (kBK * 2);
+        if constexpr (BITS == 4) {
+          uint32_t w[8];
+          const uint4 lo = *reinterpret_cast<const uint4*>(prow);
+          const uint4 hi = *reinterpret_cast<const uint4*>(prow + 16);
+          w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+          w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int gj = gin + (GS == 32 ? j / 4 : 0);  // 32-code groups: two per stage
+            const uint16_t sv = sbp[gj], bv = bbp[gj];
+            const __nv_bfloat162 s2v = __halves2bfloat162(__ushort_as_bfloat16(sv), __ushort_as_bfloat16(sv));
+            const __nv_bfloat162 b2v = __halves2bfloat162(__ushort_as_bfloat16(bv), __ushort_as_bfloat16(bv));
+            const uint4 o = dequant_word4(w[j], s2v, b2v);
+            *reinterpret_cast<uint4*>(brow + ((j ^ (row & 7)) << 4)) = o;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = codes 8c .. 8c+7 = two words
+            const uint2 ww = *reinterpret_cast<const uint2*>(prow + 8 * c);
+            const int gj = gin + (GS == 32 ? c / 4 : 0);
+            const float sv = bf16_to_f32(sbp[gj]), bv = bf16_to_f32(bbp[gj]);
+            const uint2 a = dequant_word8(ww.x, sv, bv);
+            const uint2 b = dequant_word8(ww.y, sv, bv);
+            *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+          }
+        }
+        fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&full2[s2]);
+          mbar_arrive(&empty1[s1]);
+          if (ks % KS_SB == KS_SB - 1 || ks == KS - 1) mbar_arrive(&empty_sb[e]);
+        }
+        if (ks % KS_SB == KS_SB - 1 || ks == KS - 1) ++sbit;
+      }
+      if (*abort_flag) break;
+    }
+  } else if (warp < kEpiWarps) {
+    // ------------------------------------------------------------------ epilogue
+    const int row = warp * 32 + lane;  // TMEM lane
+    uint32_t tc = 0;
+    for (int64_t u = u_begin; u < u_end; ++u, ++tc) {
+      if (*abort_flag) break;
+      const uint32_t buf = tc & 1;
+      if (!mbar_wait(&tfull[buf], (tc >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const Tile tl = tc_tile(p, u / NBLK);
+      const int64_t n0 = (u % NBLK) * unit_n;
+      const bool valid = static_cast<uint32_t>(row) < tl.valid;
+      uint16_t* yrow = nullptr;
+      if (valid) {
+        const uint32_t pos = tl.row_start + row;
+        const uint32_t dr = p.dst_row ? p.dst_row[pos] : pos;
+        yrow = p.y + static_cast<int64_t>(dr) * p.N;
+      }
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + buf * (2 * kBN);
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        float v0[32], v1[32];
+        tmem_ld32(tbase + c * 32, v0);
+        tmem_ld32(tbase + kBN + c * 32, v1);
+        if (!valid) continue;
+        if (p.pair) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int64_t nb = n0 + half * kBN + c * 32;
+            const float* v = half ? v1 : v0;
+            if (nb + 32 <= p.N && (p.N & 7) == 0) {  // 16-byte aligned row segments
+              uint4* dst = reinterpret_cast<uint4*>(yrow + nb);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_uint4(bf16x2_of(v[8 * q], v[8 * q + 1]), bf16x2_of(v[8 * q + 2], v[8 * q + 3]),
+                                    bf16x2_of(v[8 * q + 4], v[8 * q + 5]), bf16x2_of(v[8 * q + 6], v[8 * q + 7]));
+            } else {
+              for (int i = 0; i < 32 && nb + i < p.N; ++i) yrow[nb + i] = f32_to_bf16(v[i]);
+            }
+          }
+        } else {
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[i] = v0[i] * (v1[i] / (1.0f + expf(-v1[i])));
+          const int64_t nb = n0 + c * 32;
+          if (nb + 32 <= p.N && (p.N & 7) == 0) {  // 16-byte aligned row segments
+            uint4* dst = reinterpret_cast<uint4*>(yrow + nb);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(bf16x2_of(h[8 * q], h[8 * q + 1]), bf16x2_of(h[8 * q + 2], h[8 * q + 3]),
+                                  bf16x2_of(h[8 * q + 4], h[8 * q + 5]), bf16x2_of(h[8 * q + 6], h[8 * q + 7]));
+          } else {
+            for (int i = 0; i < 32 && nb + i < p.N; ++i) yrow[nb + i] = f32_to_bf16(h[i]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  // ------------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+  if (threadIdx.x == 0) prof_end(p.prof);
+}
+
+template <int BITS, int GS>
+cudaError_t launch_tc(TcParams prm, cudaStream_t stream) {
+  using C = TcCfg<BITS>;
+  auto kern = qmm_tc_kernel<BITS, GS>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::SMEM + 1024);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  LaunchTimer timer(prm.pair ? "tc" : "tc_glu", stream);
+  prm.prof = timer.slot();
+  kern<<<sm_count(), kThreads, C::SMEM + 1024, stream>>>(prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool qmm_tc_supported(const GemmArgs& a) {
+  if (a.bits != 4 && a.bits != 8) return false;
+  if (a.K % kBK != 0) return false;
+  if ((a.K / a.group) % kSbGroups != 0) return false;  // scale/bias rows: 16-byte pitch
+  if (a.x_rows <= 0) return false;
+  return true;
+}
+
+cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream) {
+  if (!qmm_tc_supported(a)) return cudaErrorNotSupported;
+  TcParams prm{};
+  cudaError_t e = make_tmap_2d_bf16(&prm.tm_a, a.x, a.K, a.x_rows, kBK, kBM, /*swizzle128=*/true);
+  if (e != cudaSuccess) return e;
+  prm.pair = a.nmat == 2 ? 0 : 1;
+  const int64_t words = a.K * a.bits / 32;
+  const int64_t gpr = a.K / a.group;
+  for (int m = 0; m < 2; ++m) {
+    const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
+    e = make_tmap_2d_u32(&prm.tm_w[m], wm.codes, words, a.E * a.N, kBK * a.bits / 32, kBM,
+                         /*swizzle128=*/false);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d_bf16(&prm.tm_sb[m][0], wm.scales, gpr, a.E * a.N, kSbGroups, kBM, false);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d_bf16(&prm.tm_sb[m][1], wm.biases, gpr, a.E * a.N, kSbGroups, kBM, false);
+    if (e != cudaSuccess) return e;
+  }
+  prm.y = a.y;
+  prm.dst_row = a.dst_row;
+  prm.tiles = a.tiles;
+  prm.num_tiles = a.num_tiles;
+  prm.dense_rows = a.dense_rows;
+  prm.N = a.N;
+  prm.K = a.K;
+  prm.d_status = a.d_status;
+  if (a.bits == 4) {
+    if (a.group == 32) return launch_tc<4, 32>(prm, stream);
+    if (a.group == 64) return launch_tc<4, 64>(prm, stream);
+    return launch_tc<4, 128>(prm, stream);
+  }
+  if (a.group == 32) return launch_tc<8, 32>(prm, stream);
+  if (a.group == 64) return launch_tc<8, 64>(prm, stream);
+  return launch_tc<8, 128>(prm, stream);
+}
 
 }  // namespace qmoe

@@ -39,3 +39,25 @@ def test_timing_slots_eager_and_graph(gpu_lib):
             assert n == 1 and 0.0 < ms < 50.0
     finally:
         q.qmoe_timing_enable(None)
+
+
+def test_forced_kernels_really_run(gpu_lib, monkeypatch):
+    """QMOE_FORCE_KERNEL selects the streaming or the tensor-core kernel: the launch
+    records prove which one ran (so the parity tests cover both)."""
+    q = gpu_lib
+    rng = np.random.default_rng(3)
+    w, s, b = random_qweight(rng, 1, 256, 512, 64, 4)
+    args = (dev_u32(w[0]), dev_bf16(s[0]), dev_bf16(b[0]), 64, 4)
+    x = dev_bf16(normal_bf16(rng, (200, 512)))
+    slots = torch.zeros(16 * 8, dtype=torch.uint8, device="cuda")
+    for forced, name in (("qmv", "qmv"), ("tc", "tc")):
+        monkeypatch.setenv("QMOE_FORCE_KERNEL", forced)
+        q.qmoe_qmm(x, *args)  # warm-up outside timing
+        torch.cuda.synchronize()
+        q.qmoe_timing_enable(slots)
+        try:
+            q.qmoe_qmm(x, *args)
+            torch.cuda.synchronize()
+            assert q.qmoe_timing_read(name)[1] == 1, forced
+        finally:
+            q.qmoe_timing_enable(None)
