@@ -245,6 +245,59 @@ CONFIG = {
 }
 
 
+def run_prefill(q, token_counts, dev, peaks, reps=5):
+    """Prefill MoE layer (Zipf-skewed routing, expert-sorted SwitchGLU, combine) at each
+    token count: layer time, TFLOP/s, and the per-kernel split from the launch timing
+    slots."""
+    import torch
+    from gpu_util import dev_bf16, dev_f32, dev_u32, qweight
+    from inputs import prefill_layer
+    out = {}
+    for T in token_counts:
+        d = prefill_layer(0, T)
+        Wp = [qweight(*d[k], GROUP, BITS) for k in ("up", "gate", "down")]
+        xp, ip, sp = dev_bf16(d["x"]), dev_u32(d["idx"]), dev_f32(d["scores"])
+        wsp = torch.empty(q.qmoe_switch_glu_workspace_size(T, TOP_K, *Wp), dtype=torch.uint8,
+                          device=dev)
+        ysp = torch.empty((T * TOP_K, 2048), dtype=torch.bfloat16, device=dev)
+        invp = torch.empty(T * TOP_K, dtype=torch.int32, device=dev)
+        outp = torch.empty((T, 2048), dtype=torch.bfloat16, device=dev)
+
+        def pf():
+            q.qmoe_switch_glu(xp, ip, *Wp, mode=1, out=ysp, inv_order=invp, workspace=wsp)
+            q.qmoe_moe_combine(ysp, invp, sp, out=outp)
+
+        for _ in range(3):
+            pf()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            pf()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / reps
+        slots = torch.zeros(16 * 64, dtype=torch.uint8, device=dev)
+        q.qmoe_timing_enable(slots)
+        pf()
+        torch.cuda.synchronize()
+        split = {k: q.qmoe_timing_read(k)[0] for k in
+                 ("route", "gather_rows", "tc_glu", "tc", "qmv_glu", "qmv", "combine")}
+        q.qmoe_timing_enable(None)
+        flop = T * TOP_K * PREFILL_FLOP_PER_ROW
+        tf = flop / (t * 1e-3) / 1e12
+        bf16_peak = peaks["bf16_tflops"] if peaks else 1590.0
+        glu_ms = split["tc_glu"] or split["qmv_glu"]
+        dn_ms = split["tc"] or split["qmv"]
+        glu_tf = T * TOP_K * 4 * 2048 * 512 / (glu_ms * 1e-3) / 1e12 if glu_ms else None
+        dn_tf = T * TOP_K * 2 * 2048 * 512 / (dn_ms * 1e-3) / 1e12 if dn_ms else None
+        out[f"T{T}"] = {"ms": t, "tflops": tf, "frac_bf16_peak": tf / bf16_peak,
+                        "kernel_ms": split, "upgate_tflops": glu_tf, "down_tflops": dn_tf}
+        del Wp, d
+    return out
+
+
 # ---------------------------------------------------------------------- ours
 def main():
     p = argparse.ArgumentParser()
@@ -256,6 +309,10 @@ def main():
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--experts", type=int, default=E,
                    help="number of experts (smaller for profiling captures)")
+    p.add_argument("--prefill-only", type=int, default=0, metavar="T",
+                   help="only time the prefill MoE layer at T tokens (profiling captures)")
+    p.add_argument("--prefill-tokens", default="4096,16384",
+                   help="comma-separated token counts of the prefill measurement")
     args = p.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, ws, local = dist_setup(args.gpus)
@@ -271,6 +328,10 @@ def main():
     q.load()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    peaks = measured_peaks()
+    if args.prefill_only:
+        print(json.dumps({"prefill": run_prefill(q, [args.prefill_only], dev, peaks)}), flush=True)
+        return
     weights = decode_weights(0, E=args.experts)
     W = [qweight(*t, GROUP, BITS) for t in weights]
 
@@ -364,7 +425,6 @@ def main():
     q.qmoe_timing_enable(None)
     del g_timed
     k_ms, k_n = sums["qmv_glu"], counts["qmv_glu"]
-    peaks = measured_peaks()
     hbm_peak = peaks["hbm_gbs"] if peaks else 6650.0
     achieved = ug_bytes / (k_ms * 1e-3) / 1e9 if k_ms > 0 else None
     roofline = {
@@ -458,36 +518,8 @@ def main():
     # prefill MoE layer (routed experts, expert-sorted, combine)
     prefill = None
     if not args.no_prefill:
-        prefill = {}
-        for T in (4096,):
-            d = prefill_layer(0, T)
-            Wp = [qweight(*d[k], GROUP, BITS) for k in ("up", "gate", "down")]
-            xp, ip, sp = dev_bf16(d["x"]), dev_u32(d["idx"]), dev_f32(d["scores"])
-            wsp = torch.empty(q.qmoe_switch_glu_workspace_size(T, TOP_K, *Wp), dtype=torch.uint8,
-                              device=dev)
-            ysp = torch.empty((T * TOP_K, 2048), dtype=torch.bfloat16, device=dev)
-            invp = torch.empty(T * TOP_K, dtype=torch.int32, device=dev)
-            outp = torch.empty((T, 2048), dtype=torch.bfloat16, device=dev)
-
-            def pf():
-                q.qmoe_switch_glu(xp, ip, *Wp, mode=1, out=ysp, inv_order=invp, workspace=wsp)
-                q.qmoe_moe_combine(ysp, invp, sp, out=outp)
-
-            for _ in range(3):
-                pf()
-            torch.cuda.synchronize()
-            reps = 5
-            e0.record(stream)
-            for _ in range(reps):
-                pf()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            t = e0.elapsed_time(e1) / reps
-            flop = T * TOP_K * PREFILL_FLOP_PER_ROW
-            tf = flop / (t * 1e-3) / 1e12
-            bf16_peak = peaks["bf16_tflops"] if peaks else 1590.0
-            prefill[f"T{T}"] = {"ms": t, "tflops": tf, "frac_bf16_peak": tf / bf16_peak}
-            del Wp, d
+        prefill = run_prefill(q, [int(t) for t in args.prefill_tokens.split(",") if t], dev,
+                              peaks)
 
     # CPU oracle on a bounded sample (rank 0, N = 1)
     cpu = None

@@ -38,7 +38,6 @@ namespace {
 constexpr int kBM = 128;            // rows per tile = TMEM lanes
 constexpr int kBN = 128;            // output channels per accumulator
 constexpr int kBK = 64;             // k per stage: one 128-byte swizzle atom of bf16
-constexpr int kS1 = 4;              // activation + packed-code ring
 constexpr int kS2 = 2;              // dequantised-weight ring
 constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps = 8;
 constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;  // 448
@@ -47,17 +46,19 @@ constexpr int kSbGroups = 8;        // groups per scale/bias TMA box (16 bytes o
 
 template <int BITS>
 struct TcCfg {
+  static constexpr int S1 = BITS == 4 ? 5 : 4;                   // activation + packed-code ring
   static constexpr int A_BYTES = kBM * kBK * 2;                  // 16 KB
   static constexpr int P_ROW = kBK * BITS / 8;                   // packed bytes per row per stage
   static constexpr int P_BYTES = 2 * kBM * P_ROW;                // two stacks
   static constexpr int B_BYTES = 2 * kBN * kBK * 2;              // two stacks, bf16
   static constexpr int SB_BYTES = 2 * 2 * kBM * kSbGroups * 2;   // [stack][s|b][row][8]
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_P = OFF_A + kS1 * A_BYTES;
-  static constexpr int OFF_B = OFF_P + kS1 * P_BYTES;
+  static constexpr int OFF_P = OFF_A + S1 * A_BYTES;
+  static constexpr int OFF_B = OFF_P + S1 * P_BYTES;
   static constexpr int OFF_SB = OFF_B + kS2 * B_BYTES;
   static constexpr int OFF_BAR = OFF_SB + 2 * SB_BYTES;
   static constexpr int SMEM = OFF_BAR + 256;
+  static_assert(SMEM + 1024 <= 227 * 1024, "shared memory budget");
   static_assert(OFF_P % 1024 == 0 && OFF_B % 1024 == 0 && OFF_SB % 1024 == 0, "alignment");
 };
 
@@ -194,6 +195,7 @@ __device__ __forceinline__ uint2 dequant_word8(uint32_t w, float s, float b) {
 template <int BITS, int GS>
 __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<BITS>;
+  constexpr int kS1 = C::S1;
   // stages covered by one scale/bias box of kSbGroups groups
   constexpr int KS_SB = kSbGroups * GS / kBK;
   static_assert(KS_SB >= 1 && (kSbGroups * GS) % kBK == 0, "group size");
@@ -247,9 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
   const int unit_n = p.pair ? 2 * kBN : kBN;
   const int64_t NBLK = (p.N + unit_n - 1) / unit_n;
   const int64_t ntiles = p.dense_rows > 0 ? (p.dense_rows + kBM - 1) / kBM : *p.num_tiles;
+  // Units are dealt round-robin: at any moment the CTAs work on consecutive units, so
+  // the channel blocks of one activation tile (and the tiles of one expert) run
+  // concurrently and share their operands through L2.
   const int64_t units = ntiles * NBLK;
-  const int64_t u_begin = units * blockIdx.x / gridDim.x;
-  const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
+  const int64_t u_begin = blockIdx.x, u_step = gridDim.x;
+  const int64_t u_end = units;
 
   if (warp == kProdWarp) {
     // ------------------------------------------------------------------ producer
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
       tma_prefetch_desc(&p.tm_a);
       uint32_t it = 0, sbit = 0;
       bool ab = false;
-      for (int64_t u = u_begin; u < u_end && !ab; ++u) {
+      for (int64_t u = u_begin; u < u_end && !ab; u += u_step) {
         const Tile tl = tc_tile(p, u / NBLK);
         const int64_t n0 = (u % NBLK) * unit_n;
         const int64_t wrow = static_cast<int64_t>(tl.expert) * p.N + n0;
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     if (lane == 0) {
       uint32_t it = 0, tc = 0;
       bool issued = false;
-      for (int64_t u = u_begin; u < u_end; ++u, ++tc) {
+      for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
         if (*abort_flag) break;
         const uint32_t buf = tc & 1;
         if (!mbar_wait(&tempty[buf], ((tc >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
@@ -344,10 +349,13 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     }
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------------------------------- dequant
+    // Thread dq handles half-rows hr = dq and dq + 256 of the 512 (stack, row, half)
+    // half-rows of a stage: consecutive lanes read consecutive 16-byte pieces of the
+    // packed tile and write distinct swizzled 16-byte chunks (no bank conflicts).
     const int dq = threadIdx.x - kDqWarp0 * 32;  // 0..255
-    const int m = dq / kBM, row = dq % kBM;
+    constexpr int HALF = C::P_ROW / 2;           // packed bytes per half-row: 16 or 32
     uint32_t it = 0, sbit = 0;
-    for (int64_t u = u_begin; u < u_end; ++u) {
+    for (int64_t u = u_begin; u < u_end; u += u_step) {
       for (int64_t ks = 0; ks < KS; ++ks, ++it) {
         if (*abort_flag) break;
         const uint32_t e = sbit & 1;
@@ -356,36 +364,41 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         const uint32_t s1 = it % kS1, s2 = it % kS2;
         if (!mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) ||
             !mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
-        const uint16_t* sbp = reinterpret_cast<const uint16_t*>(smem + C::OFF_SB + e * C::SB_BYTES) +
-                              ((m * 2) * kBM + row) * kSbGroups;
-        const uint16_t* bbp = sbp + kBM * kSbGroups;
         const int gin = static_cast<int>((ks * kBK / GS) % kSbGroups);
-        const uint8_t* prow = smem + C::OFF_P + s1 * C::P_BYTES + (m * kBM + row) * C::P_ROW;
-        uint8_t* brow = smem + C::OFF_B + s2 * C::B_BYTES + (m * kBN + row) * (kBK * 2);
-        if constexpr (BITS == 4) {
-          uint32_t w[8];
-          const uint4 lo = *reinterpret_cast<const uint4*>(prow);
-          const uint4 hi = *reinterpret_cast<const uint4*>(prow + 16);
-          w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
-          w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int gj = gin + (GS == 32 ? j / 4 : 0);  // 32-code groups: two per stage
+        for (int rep = 0; rep < 2; ++rep) {
+          const int hr = dq + 256 * rep;          // (stack, row, half)
+          const int m = hr / (2 * kBM), row = (hr / 2) % kBM, half = hr & 1;
+          const uint16_t* sbp = reinterpret_cast<const uint16_t*>(smem + C::OFF_SB + e * C::SB_BYTES) +
+                                ((m * 2) * kBM + row) * kSbGroups;
+          const uint16_t* bbp = sbp + kBM * kSbGroups;
+          const uint8_t* prow = smem + C::OFF_P + s1 * C::P_BYTES + (m * kBM + row) * C::P_ROW + half * HALF;
+          uint8_t* brow = smem + C::OFF_B + s2 * C::B_BYTES + (m * kBN + row) * (kBK * 2);
+          // codes 32*half .. 32*half+31 of this row's 64
+          const int gj = gin + (GS == 32 ? half : 0);
+          if constexpr (BITS == 4) {
+            const uint4 pw = *reinterpret_cast<const uint4*>(prow);
+            const uint32_t w[4] = {pw.x, pw.y, pw.z, pw.w};
             const uint16_t sv = sbp[gj], bv = bbp[gj];
             const __nv_bfloat162 s2v = __halves2bfloat162(__ushort_as_bfloat16(sv), __ushort_as_bfloat16(sv));
             const __nv_bfloat162 b2v = __halves2bfloat162(__ushort_as_bfloat16(bv), __ushort_as_bfloat16(bv));
-            const uint4 o = dequant_word4(w[j], s2v, b2v);
-            *reinterpret_cast<uint4*>(brow + ((j ^ (row & 7)) << 4)) = o;
-          }
-        } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = codes 8c .. 8c+7 = two words
-            const uint2 ww = *reinterpret_cast<const uint2*>(prow + 8 * c);
-            const int gj = gin + (GS == 32 ? c / 4 : 0);
+            for (int j = 0; j < 4; ++j) {
+              const int c = 4 * half + j;             // 16-byte chunk = codes 8c .. 8c+7
+              *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = dequant_word4(w[j], s2v, b2v);
+            }
+          } else {
+            const uint4 pa = *reinterpret_cast<const uint4*>(prow);
+            const uint4 pb = *reinterpret_cast<const uint4*>(prow + 16);
+            const uint32_t w[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
             const float sv = bf16_to_f32(sbp[gj]), bv = bf16_to_f32(bbp[gj]);
-            const uint2 a = dequant_word8(ww.x, sv, bv);
-            const uint2 b = dequant_word8(ww.y, sv, bv);
-            *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int c = 4 * half + j;             // two 8-bit words per chunk
+              const uint2 a = dequant_word8(w[2 * j], sv, bv);
+              const uint2 b = dequant_word8(w[2 * j + 1], sv, bv);
+              *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+            }
           }
         }
         fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
@@ -403,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     // ------------------------------------------------------------------ epilogue
     const int row = warp * 32 + lane;  // TMEM lane
     uint32_t tc = 0;
-    for (int64_t u = u_begin; u < u_end; ++u, ++tc) {
+    for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
       if (*abort_flag) break;
       const uint32_t buf = tc & 1;
       if (!mbar_wait(&tfull[buf], (tc >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
