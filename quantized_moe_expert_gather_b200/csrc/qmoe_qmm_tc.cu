@@ -455,7 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         } else {
           float h[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) h[i] = v0[i] * (v1[i] / (1.0f + expf(-v1[i])));
+          for (int i = 0; i < 32; ++i)
+            h[i] = v0[i] * v1[i] * __frcp_rn(1.0f + __expf(-v1[i]));  // up * silu(gate)
           const int64_t nb = n0 + c * 32;
           if (nb + 32 <= p.N && (p.N & 7) == 0) {  // 16-byte aligned row segments
             uint4* dst = reinterpret_cast<uint4*>(yrow + nb);
