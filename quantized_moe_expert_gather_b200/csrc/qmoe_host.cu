@@ -44,6 +44,21 @@ cudaError_t make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int esize, const
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+
+cudaError_t make_tmap_colblocks(CUtensorMap* map, const void* base, int64_t words, int64_t rows,
+                                int box_rows, int box_blocks) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  if (words % 32 != 0) return cudaErrorInvalidValue;
+  cuuint64_t dims[3] = {32, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(words / 32)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(words * 4), 128};
+  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_blocks)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 }  // namespace
 
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
@@ -88,6 +103,10 @@ cudaError_t make_tmap_2d_u32(CUtensorMap* map, const void* base, int64_t inner, 
                              int box_inner, int box_rows, bool swizzle128) {
   return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, base, inner, rows, box_inner,
                    box_rows, swizzle128);
+}
+cudaError_t make_tmap_3d_u32_colblocks(CUtensorMap* map, const void* base, int64_t words,
+                                       int64_t rows, int box_rows, int box_blocks) {
+  return make_tmap_colblocks(map, base, words, rows, box_rows, box_blocks);
 }
 cudaError_t make_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
                               int box_inner, int box_rows, bool swizzle128) {

@@ -9,7 +9,8 @@
 // The tile table makes every touched expert's packed weights stream from HBM once
 // per tile (MLX issue #4509: M=1 decode must still reach full bandwidth).
 //
-// Structure (one persistent CTA per SM, CW consumer warps + 1 producer warp):
+// Structure (one persistent CTA per SM, CW consumer warps + 1 producer warp + 1
+// epilogue warp):
 //   * the last warp (producer) walks the CTA's contiguous range of (tile, 16-row block)
 //     units and, per K-chunk, loads the 16 packed rows with 2-D TMA boxes of
 //     128 B x 16 rows (128B-swizzled, so the consumers' row-strided reads are free
@@ -26,7 +27,11 @@
 //     with C the MMA sum over the magic-offset codes and X = sum_k x_k, obtained
 //     from one more MMA with an all-ones A.  Scales and biases stay exact (fp32),
 //     accumulation is fp32, and there is one bf16 rounding at the end;
-//   * consumers reduce their partial sums through shared memory and write bf16.
+//   * consumers store their partial sums of a unit in per-warp shared-memory slots and
+//     move on; a dedicated epilogue warp waits for all slots (mbarrier), adds them in
+//     warp order (deterministic, and a row's result does not depend on the other rows
+//     of its tile), applies silu*mul and writes bf16.  Two slot buffers alternate, so
+//     consumers never wait for each other at unit boundaries.
 //
 // All waits are bounded (see qmoe_common.cuh).
 #include <algorithm>
@@ -55,9 +60,11 @@ constexpr int consumer_warps() {
 template <int BITS, int GS, int NMAT, int NT>
 struct Cfg {
   static constexpr int CW = consumer_warps<BITS, GS, NT>();
-  static constexpr int THREADS = (CW + 1) * 32;
+  static constexpr int THREADS = (CW + 2) * 32;  // consumers, producer, epilogue
   static constexpr int KB_BYTES = GS * BITS / 8;                 // one group of one row
-  static constexpr int CHUNK_ROW_BYTES = std::max(512, KB_BYTES * CW);
+  // 1 KB of each row per stage (512 B with two token sets, whose doubled register
+  // arrays would otherwise spill), at least one group per consumer warp
+  static constexpr int CHUNK_ROW_BYTES = std::max(NT == 2 ? 512 : 1024, KB_BYTES * CW);
   static constexpr int KB_PER_CHUNK = CHUNK_ROW_BYTES / KB_BYTES;
   static constexpr int KB_PER_WARP = KB_PER_CHUNK / CW;
   static constexpr int BOXES = CHUNK_ROW_BYTES / 128;
@@ -71,7 +78,7 @@ struct Cfg {
   static constexpr int RED_BYTES = 2 * RED_SLICE * 4;
   static constexpr int STAGES =
       std::min(8, (kSmemBudget - RED_BYTES - 1024) / STAGE_BYTES);
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RED_BYTES + 2 * STAGES * 8 + 64;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RED_BYTES + 2 * STAGES * 8 + 4 * 8 + 64;
   static constexpr uint32_t TMA_BYTES = CODE_BYTES;
   static_assert((kRows * KB_PER_CHUNK * 2) % 128 == 0, "scale/bias TMA boxes must stay 128-byte aligned");
   static constexpr float OFFSET = BITS == 4 ? 128.0f : 2176.0f;
@@ -93,6 +100,7 @@ struct alignas(64) QmvParams {
   int64_t dense_rows;
   int64_t N, K, E;
   int pair;                     // 1: one weight stack, a unit is two adjacent 16-row blocks
+  int code3d;                   // codes by one 3-D box per 16-row block (else one 2-D box per 128 B)
   int sb_tma;                   // scales/biases by TMA (row pitch a multiple of 16 bytes)
   int sb_vec;                   // else: byte width of the copy pieces (2: plain copies)
   int* d_status;
@@ -141,7 +149,9 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
   float* red = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::RED_BYTES);
   uint64_t* empty = full + C::STAGES;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::STAGES);
+  uint64_t* red_full = empty + C::STAGES;   // [2] every consumer lane has stored its partials
+  uint64_t* red_empty = red_full + 2;       // [2] the epilogue warp has read the buffer
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -149,6 +159,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
       // producer's expect_tx (+ 32 per-lane arrivals when scales/biases are copied by lanes)
       mbar_init(&full[s], p.sb_tma ? 1 : 1 + 32);
       mbar_init(&empty[s], kConsumerWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&red_full[b], kConsumerWarps * 32);
+      mbar_init(&red_empty[b], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -195,13 +209,21 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
         uint8_t* st = smem + stage * C::STAGE_BYTES;
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[stage], C::TMA_BYTES + (p.sb_tma ? C::SB_BYTES : 0u));
-          const int32_t xw = static_cast<int32_t>(ch * (C::CHUNK_ROW_BYTES / 4));
+          if (p.code3d) {
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m)
+            for (int m = 0; m < NMAT; ++m)
+              tma_load_3d(st + m * C::BOXES * 2048, &p.tmap[m], &full[stage], 0,
+                          static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)),
+                          static_cast<int32_t>(ch * C::BOXES));
+          } else {
+            const int32_t xw = static_cast<int32_t>(ch * (C::CHUNK_ROW_BYTES / 4));
 #pragma unroll
-            for (int bx = 0; bx < C::BOXES; ++bx)
-              tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[m], &full[stage], xw + bx * 32,
-                          static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+              for (int bx = 0; bx < C::BOXES; ++bx)
+                tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[m], &full[stage],
+                            xw + bx * 32, static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
+          }
           if (p.sb_tma) {
             const int32_t xg = static_cast<int32_t>(ch * C::KB_PER_CHUNK);
 #pragma unroll
@@ -253,6 +275,55 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
       for (uint32_t k = first; k < it; ++k)
         mbar_wait(&full[k % C::STAGES], (k / C::STAGES) & 1, nullptr);
     }
+    return;
+  }
+
+  if (warp == kConsumerWarps + 1) {
+    // -------------------------------------------------------------- epilogue warp
+    for (int64_t u = u_begin; u < u_end; ++u) {
+      const uint32_t ui = static_cast<uint32_t>(u - u_begin), b = ui & 1;
+      if (*abort_flag) break;
+      if (!mbar_wait(&red_full[b], (ui >> 1) & 1, p.d_status)) {
+        *abort_flag = 1;
+        break;
+      }
+      const TileInfo ti = tile_info<NT>(p, u / NB);
+      const int64_t n0 = (u % NB) * unit_rows;
+      const float* ub = red + b * C::RED_SLICE;
+      // one (token slot, row) entry per lane and pass; only the tile's valid rows
+      for (int e = lane; e < static_cast<int>(ti.valid) * kRows; e += 32) {
+        const int slot = e / kRows, row = e % kRows, nt = slot / 8, tok = slot % 8;
+        float v[NMAT];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          float sum = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w)
+            sum += ub[(((w * NMAT + m) * NT + nt) * kRows + row) * 8 + tok];
+          v[m] = sum;
+        }
+        const uint32_t pos = ti.row_start + slot;
+        const uint32_t dr = p.dst_row ? p.dst_row[pos] : pos;
+        uint16_t* yrow = p.y + static_cast<int64_t>(dr) * p.N;
+        if (p.pair) {
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            const int64_t n = n0 + kRows * m + row;
+            if (n < p.N) yrow[n] = f32_to_bf16(v[m]);
+          }
+        } else if (n0 + row < p.N) {
+          float out = v[0];
+          if constexpr (NMAT == 2) {
+            const float gte = v[1];
+            out = v[0] * (gte / (1.0f + expf(-gte)));
+          }
+          yrow[n0 + row] = f32_to_bf16(out);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_empty[b]);
+    }
+    if (lane == 0) prof_end(p.prof);  // the epilogue warp finishes the CTA's work
     return;
   }
 
@@ -459,68 +530,48 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
       if (lane == 0) mbar_arrive(&empty[stage]);
     }
 
-    // ---- cross-warp reduction: each warp stores its partial sums (valid token
-    // columns only) in its own slot; the epilogue adds the slots in warp order, so the
-    // result does not depend on timing.  Two buffers alternate between units: one
-    // barrier per unit suffices.
-    float* ub = red + ((u - u_begin) & 1) * C::RED_SLICE;
-    if (!*abort_flag) {
+    // ---- hand the partial sums to the epilogue warp (valid token columns only)
+    {
+      const uint32_t ui = static_cast<uint32_t>(u - u_begin), b = ui & 1;
+      if (ui >= 2 && !*abort_flag && !mbar_wait(&red_empty[b], ((ui >> 1) - 1) & 1, p.d_status))
+        *abort_flag = 1;
+      float* ub = red + b * C::RED_SLICE;
+      if (!*abort_flag) {
 #pragma unroll
-      for (int m = 0; m < NMAT; ++m)
+        for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float* r = ub + (((warp * NMAT + m) * NT + nt) * kRows) * 8;
+          for (int nt = 0; nt < NT; ++nt) {
+            float* r = ub + (((warp * NMAT + m) * NT + nt) * kRows) * 8;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            if (static_cast<uint32_t>(nt * 8 + 2 * t + j) < ti.valid) {
-              r[g * 8 + 2 * t + j] = acc[m][nt][j];
-              r[(g + 8) * 8 + 2 * t + j] = acc[m][nt][2 + j];
+            for (int j = 0; j < 2; ++j) {
+              if (static_cast<uint32_t>(nt * 8 + 2 * t + j) < ti.valid) {
+                r[g * 8 + 2 * t + j] = acc[m][nt][j];
+                r[(g + 8) * 8 + 2 * t + j] = acc[m][nt][2 + j];
+              }
             }
           }
-        }
-    }
-    named_bar_sync(1, kConsumerWarps * 32);
-    // ---- epilogue: one thread per (row, token) entry
-    const int tid = threadIdx.x;
-    if (tid < NT * 128) {
-      const int nt = tid / 128, rem = tid % 128, tok = rem / 16, row = rem % 16;
-      const uint32_t slot = nt * 8 + tok;
-      if (!*abort_flag && slot < ti.valid) {
-        float v[NMAT];
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-          float sum = 0.f;
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w)
-            sum += ub[(((w * NMAT + m) * NT + nt) * kRows + row) * 8 + tok];
-          v[m] = sum;
-        }
-        const uint32_t pos = ti.row_start + slot;
-        const uint32_t dr = p.dst_row ? p.dst_row[pos] : pos;
-        uint16_t* yrow = p.y + static_cast<int64_t>(dr) * p.N;
-        if (p.pair) {
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            const int64_t n = n0 + kRows * m + row;
-            if (n < p.N) yrow[n] = f32_to_bf16(v[m]);
-          }
-        } else if (n0 + row < p.N) {
-          float out = v[0];
-          if constexpr (NMAT == 2) {
-            const float gte = v[1];
-            out = v[0] * (gte / (1.0f + expf(-gte)));
-          }
-          yrow[n0 + row] = f32_to_bf16(out);
-        }
       }
+      mbar_arrive(&red_full[b]);  // release: orders this lane's stores
     }
   }
-  if (threadIdx.x == 0) prof_end(p.prof);
 }
 
 template <int BITS, int GS, int NMAT, int NT>
 cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
   using C = Cfg<BITS, GS, NMAT, NT>;
+  // Codes: one 3-D box (16 rows x BOXES column blocks of 128 B) per 16-row block when
+  // the row is a whole number of column blocks, else BOXES 2-D boxes of 128 B x 16 rows.
+  const int64_t words = a.K * a.bits / 32;
+  prm.code3d = (words % 32 == 0) ? 1 : 0;
+  for (int m = 0; m < 2; ++m) {
+    const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
+    cudaError_t e = prm.code3d
+                        ? make_tmap_3d_u32_colblocks(&prm.tmap[m], wm.codes, words, a.E * a.N,
+                                                     kRows, C::BOXES)
+                        : make_tmap_2d_u32(&prm.tmap[m], wm.codes, words, a.E * a.N, 32, kRows,
+                                           /*swizzle128=*/true);
+    if (e != cudaSuccess) return e;
+  }
   const int64_t gpr = a.K / GS;
   prm.sb_tma = (gpr % 8 == 0) ? 1 : 0;
   if (prm.sb_tma) {
@@ -560,13 +611,9 @@ cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cuda
 
 cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
   QmvParams prm{};
-  const int64_t words = a.K * a.bits / 32;
   prm.pair = a.nmat == 2 ? 0 : 1;
   for (int m = 0; m < 2; ++m) {
     const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
-    cudaError_t e = make_tmap_2d_u32(&prm.tmap[m], wm.codes, words, a.E * a.N, 32, 16,
-                                     /*swizzle128=*/true);
-    if (e != cudaSuccess) return e;
     prm.scales[m] = wm.scales;
     prm.biases[m] = wm.biases;
   }
