@@ -9,16 +9,22 @@
 // The tile table makes every touched expert's packed weights stream from HBM once
 // per tile (MLX issue #4509: M=1 decode must still reach full bandwidth).
 //
-// Structure (one persistent CTA per SM, CW consumer warps + 1 producer warp + 1
+// Structure (one persistent CTA per SM, 8 consumer warps + 1 producer warp + 1
 // epilogue warp):
-//   * the last warp (producer) walks the CTA's contiguous range of (tile, 16-row block)
-//     units and, per K-chunk, loads the 16 packed rows with 2-D TMA boxes of
-//     128 B x 16 rows (128B-swizzled, so the consumers' row-strided reads are free
-//     of bank conflicts) and the matching scales/biases with cp.async, into a ring
-//     of stages guarded by full/empty mbarriers;
+//   * the producer warp walks the CTA's contiguous range of (tile, 16-row block) units
+//     and, per K-chunk of 1 KB of each row (512 B with two token sets), loads each
+//     16-row block's packed codes with one 3-D TMA box (16 rows x 8 column blocks of
+//     128 B, 128B-swizzled so that the
+//     consumers' row-strided reads are free of bank conflicts; eight 2-D boxes of
+//     128 B x 16 rows when a row is not a whole number of column blocks) and the
+//     matching scales/biases with 2-D TMA boxes (cp.async when their row pitch is not
+//     a multiple of 16 bytes), into a ring of stages guarded by full/empty mbarriers.
+//     Few large copies per stage matter: the TMA issue and mbarrier round trip of
+//     each copy, not DRAM, bounded the stream when every 2 KB box was its own copy;
 //   * warps 0..CW-1 (consumers) split each chunk's groups.  Each lane prefetches the
 //     activation values its MMA fragments need one chunk ahead into registers (the
-//     loads of chunk c+1 are in flight while chunk c is computed).  A lane turns its packed
+//     loads of chunk c+1 are in flight while chunk c is computed; two register buffers
+//     alternate between consecutive chunks).  A lane turns its packed
 //     codes into bf16 "128 + q" (or "2048 + 16*hi" for the high nibble of 8-bit
 //     codes) with one LOP3 per code pair and feeds mma.sync m16n8k16 with W as the
 //     16-row A operand and up to 8 routed rows as the B operand.  Each MMA k-step
@@ -50,11 +56,13 @@ namespace {
 constexpr int kRows = 16;             // output channels per unit (MMA M)
 constexpr int kSmemBudget = 225 * 1024;
 
-// Consumer warps: 16 where the register budget allows (more warps hide the shared
-// memory and MMA latencies of the streaming loop), else 8.
+// Consumer warps: 8.  With the producer and epilogue warps that is 10 warps (three
+// per scheduler), which leaves each thread 168 registers: room for two chunks of
+// activations and several groups' MMA chains in flight per warp.  More warps cap the
+// registers at 96 (five warps on some schedulers) and spill.
 template <int BITS, int GS, int NT>
 constexpr int consumer_warps() {
-  return (BITS == 4 && NT == 1 && GS <= 64) ? 16 : 8;
+  return 8;
 }
 
 template <int BITS, int GS, int NMAT, int NT>
@@ -331,11 +339,33 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
   const int g = lane >> 2, t = lane & 3;
   const uint32_t ONES = 0x3F803F80u;  // bf16x2 (1, 1)
   // Activation values of one chunk for this lane: [k-block][token set][word]; 16 B per
-  // 4-bit word (8 codes), 8 B per 8-bit word (4 codes).
+  // 4-bit word (8 codes), 8 B per 8-bit word (4 codes).  Two buffers alternate: one is
+  // consumed while the loads of the next chunk land in the other.
   using XV = typename std::conditional<BITS == 4, uint4, uint2>::type;
-  XV xc[C::KB_PER_WARP][NT][C::WORDS], xn[C::KB_PER_WARP][NT][C::WORDS];
+  using XBuf = XV[C::KB_PER_WARP][NT][C::WORDS];
+  XBuf xa, xb;
 
-  // Row pointers of this lane's token slots for unit u (null for empty slots).
+  // Shared-memory offsets of this lane, fixed for the kernel.  The warp's group i sits
+  // CW*KB_BYTES bytes further along the chunk row: whole 128-byte column blocks, so
+  // GROUP_STEP bytes further in the stage with the same swizzle phase.  Row g+8 sits
+  // 1024 bytes after row g (same phase: the swizzle uses the row's low three bits).
+  constexpr int GROUP_STRIDE = C::CW * C::KB_BYTES;
+  static_assert(GROUP_STRIDE % 128 == 0, "a warp's groups must lie whole column blocks apart");
+  constexpr uint32_t GROUP_STEP = GROUP_STRIDE / 128 * 2048;
+  constexpr int PIECES = C::LANE_BYTES >= 16 ? C::LANE_BYTES / 16 : 1;
+  uint32_t code_off[PIECES];
+#pragma unroll
+  for (int q = 0; q < PIECES; ++q)
+    code_off[q] = swz(g, warp * C::KB_BYTES + t * C::LANE_BYTES + 16 * q);
+  const int sb_off = g * C::KB_PER_CHUNK + warp;  // into each [16 rows][KB_PER_CHUNK] array
+  const int x_off = warp * GS + t * (GS / 4);     // the lane's first activation of a chunk
+  constexpr int64_t CHUNK_ELEMS = static_cast<int64_t>(C::KB_PER_CHUNK) * GS;
+
+  // groups of chunk ch that lie inside [0, K/GS)
+  auto chunk_groups = [&](int64_t ch) -> int {
+    return static_cast<int>(imin64(C::KB_PER_CHUNK, KB_TOTAL - ch * C::KB_PER_CHUNK));
+  };
+  // This lane's activation pointers for unit u (null for empty token slots).
   auto tile_rows = [&](int64_t u, TileInfo& ti, const uint16_t* (&rows)[NT]) {
     ti = tile_info<NT>(p, u / NB);
 #pragma unroll
@@ -345,213 +375,240 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
       if (slot < ti.valid) {
         const uint32_t pos = ti.row_start + slot;
         const uint32_t sr = p.src_row ? p.src_row[pos] : pos;
-        rows[nt] = p.x + static_cast<int64_t>(sr) * p.K;
+        rows[nt] = p.x + static_cast<int64_t>(sr) * p.K + x_off;
       }
     }
   };
   // Issues the loads of chunk `ch` for the given rows into `dst`.
-  auto load_x = [&](const uint16_t* const (&rows)[NT], int64_t ch, XV (&dst)[C::KB_PER_WARP][NT][C::WORDS]) {
+  auto load_x = [&](const uint16_t* const (&rows)[NT], int64_t ch, XBuf& dst) {
+    const int nkb = chunk_groups(ch);
 #pragma unroll
     for (int i = 0; i < C::KB_PER_WARP; ++i) {
-      const int64_t kb = ch * C::KB_PER_CHUNK + warp + kConsumerWarps * i;
-      const int64_t k0 = kb * GS + t * (GS / 4);
+      const bool live = warp + C::CW * i < nkb;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int j = 0; j < C::WORDS; ++j) {
           if constexpr (BITS == 4) {
             dst[i][nt][j] = make_uint4(0, 0, 0, 0);
-            if (rows[nt] != nullptr && kb < KB_TOTAL) dst[i][nt][j] = ldg_nc_v4(rows[nt] + k0 + 8 * j);
+            if (rows[nt] != nullptr && live)
+              dst[i][nt][j] = ldg_nc_v4(rows[nt] + ch * CHUNK_ELEMS + i * C::CW * GS + 8 * j);
           } else {
             dst[i][nt][j] = make_uint2(0, 0);
-            if (rows[nt] != nullptr && kb < KB_TOTAL) dst[i][nt][j] = ldg_nc_v2(rows[nt] + k0 + 4 * j);
+            if (rows[nt] != nullptr && live)
+              dst[i][nt][j] = ldg_nc_v2(rows[nt] + ch * CHUNK_ELEMS + i * C::CW * GS + 4 * j);
           }
         }
     }
   };
 
+  int64_t u = u_begin, ch = 0;
   uint32_t it = 0;
-  TileInfo ti_next{};
+  TileInfo ti{}, ti_next{};
+  const uint16_t* rows[NT];
   const uint16_t* rows_next[NT];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) rows_next[nt] = nullptr;
-  if (u_begin < u_end) {
-    tile_rows(u_begin, ti_next, rows_next);
-    load_x(rows_next, 0, xn);
-  }
-  for (int64_t u = u_begin; u < u_end; ++u) {
-    const TileInfo ti = ti_next;
-    const uint16_t* rows[NT];
+  for (int nt = 0; nt < NT; ++nt) rows[nt] = rows_next[nt] = nullptr;
+  float acc[NMAT][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) rows[nt] = rows_next[nt];
-    const int64_t n0 = (u % NB) * unit_rows;
-    if (u + 1 < u_end) tile_rows(u + 1, ti_next, rows_next);  // one unit ahead
-    float acc[NMAT][NT][4];
+  for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.f;
+  if (u_begin < u_end) {
+    tile_rows(u_begin, ti, rows);
+    if (u_begin + 1 < u_end) tile_rows(u_begin + 1, ti_next, rows_next);
+    load_x(rows, 0, xa);
+  }
+
+  // Hands the partial sums of unit u to the epilogue warp (valid token columns only).
+  auto finish_unit = [&]() {
+    const uint32_t ui = static_cast<uint32_t>(u - u_begin), b = ui & 1;
+    if (ui >= 2 && !*abort_flag && !mbar_wait(&red_empty[b], ((ui >> 1) - 1) & 1, p.d_status))
+      *abort_flag = 1;
+    float* ub = red + b * C::RED_SLICE;
+    if (!*abort_flag) {
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float* r = ub + (((warp * NMAT + m) * NT + nt) * kRows) * 8;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (static_cast<uint32_t>(nt * 8 + 2 * t + j) < ti.valid) {
+              r[g * 8 + 2 * t + j] = acc[m][nt][j];
+              r[(g + 8) * 8 + 2 * t + j] = acc[m][nt][2 + j];
+            }
+          }
+        }
+    }
+    mbar_arrive(&red_full[b]);  // release: orders this lane's stores
 #pragma unroll
     for (int m = 0; m < NMAT; ++m)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.f;
+  };
 
-    for (int64_t ch = 0; ch < NCH; ++ch, ++it) {
-      // take this chunk's activations; start the next chunk's loads
+  // One chunk: its activations are in xc; the next chunk's loads go to xn.
+  auto step = [&](XBuf& xc, XBuf& xn) {
+    if (ch + 1 < NCH)
+      load_x(rows, ch + 1, xn);
+    else if (u + 1 < u_end)
+      load_x(rows_next, 0, xn);
+    const int nkb = chunk_groups(ch);
+    const int stage = it % C::STAGES;
+    bool ok = false;
+    if (!*abort_flag) {
+      ok = mbar_wait(&full[stage], (it / C::STAGES) & 1, p.d_status);
+      if (!ok) *abort_flag = 1;
+    }
+    if (ok) {
+      const uint8_t* st = smem + stage * C::STAGE_BYTES;
+      const uint16_t* sb = reinterpret_cast<const uint16_t*>(st + C::CODE_BYTES) + sb_off;
+#pragma unroll
+      for (int i = 0; i < C::KB_PER_WARP; ++i) {
+        if (warp + C::CW * i >= nkb) break;
+        // ---- B operand: x values of this lane's codes, permuted to the MMA k order
+        uint32_t bfr[NT][C::WORDS][2][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int j = 0; j < C::WORDS; ++j) {
+            if constexpr (BITS == 4) {
+              const uint4 v = xc[i][nt][j];
+              bfr[nt][j][0][0] = prmt(v.x, v.z, 0x5410);
+              bfr[nt][j][0][1] = prmt(v.x, v.z, 0x7632);
+              bfr[nt][j][1][0] = prmt(v.y, v.w, 0x5410);
+              bfr[nt][j][1][1] = prmt(v.y, v.w, 0x7632);
+            } else {
+              const uint2 v = xc[i][nt][j];
+              bfr[nt][j][0][0] = prmt(v.x, v.y, 0x5410);
+              bfr[nt][j][0][1] = prmt(v.x, v.y, 0x7632);
+              bfr[nt][j][1][0] = bfr[nt][j][0][0];
+              bfr[nt][j][1][1] = bfr[nt][j][0][1];
+            }
+          }
+        }
+        // ---- X = sum of x over the group (all-ones A operand)
+        float cx[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int i2 = 0; i2 < 4; ++i2) cx[nt][i2] = 0.f;
+          const uint32_t ones[4] = {ONES, ONES, ONES, ONES};
+#pragma unroll
+          for (int j = 0; j < C::WORDS; ++j) {
+            mma_bf16_16816(cx[nt], ones, bfr[nt][j][0][0], bfr[nt][j][0][1]);
+            if constexpr (BITS == 4) mma_bf16_16816(cx[nt], ones, bfr[nt][j][1][0], bfr[nt][j][1][1]);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          const uint8_t* cm = st + m * C::BOXES * 2048 + i * GROUP_STEP;
+          uint32_t wg[C::WORDS], wg8[C::WORDS];
+          if constexpr (C::LANE_BYTES == 4) {
+            wg[0] = *reinterpret_cast<const uint32_t*>(cm + code_off[0]);
+            wg8[0] = *reinterpret_cast<const uint32_t*>(cm + code_off[0] + 1024);
+          } else if constexpr (C::LANE_BYTES == 8) {
+            const uint2 a = *reinterpret_cast<const uint2*>(cm + code_off[0]);
+            const uint2 b = *reinterpret_cast<const uint2*>(cm + code_off[0] + 1024);
+            wg[0] = a.x; wg[1] = a.y; wg8[0] = b.x; wg8[1] = b.y;
+          } else {
+#pragma unroll
+            for (int q = 0; q < PIECES; ++q) {
+              const uint4 a = *reinterpret_cast<const uint4*>(cm + code_off[q]);
+              const uint4 b = *reinterpret_cast<const uint4*>(cm + code_off[q] + 1024);
+              wg[4 * q + 0] = a.x; wg[4 * q + 1] = a.y; wg[4 * q + 2] = a.z; wg[4 * q + 3] = a.w;
+              wg8[4 * q + 0] = b.x; wg8[4 * q + 1] = b.y; wg8[4 * q + 2] = b.z; wg8[4 * q + 3] = b.w;
+            }
+          }
+          float cacc[NT][4];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i2 = 0; i2 < 4; ++i2) cacc[nt][i2] = 0.f;
+#pragma unroll
+          for (int j = 0; j < C::WORDS; ++j) {
+            uint32_t a[2][4];
+            if constexpr (BITS == 4) {
+              const uint32_t M4 = 0x000F000Fu, MAG = 0x43004300u;
+              a[0][0] = and_or(wg[j], M4, MAG);
+              a[0][1] = and_or(wg8[j], M4, MAG);
+              a[0][2] = and_or(wg[j] >> 4, M4, MAG);
+              a[0][3] = and_or(wg8[j] >> 4, M4, MAG);
+              a[1][0] = and_or(wg[j] >> 8, M4, MAG);
+              a[1][1] = and_or(wg8[j] >> 8, M4, MAG);
+              a[1][2] = and_or(wg[j] >> 12, M4, MAG);
+              a[1][3] = and_or(wg8[j] >> 12, M4, MAG);
+            } else {
+              const uint32_t M4 = 0x000F000Fu, LO = 0x43004300u, HI = 0x45004500u;
+              a[0][0] = and_or(wg[j], M4, LO);
+              a[0][1] = and_or(wg8[j], M4, LO);
+              a[0][2] = and_or(wg[j] >> 8, M4, LO);
+              a[0][3] = and_or(wg8[j] >> 8, M4, LO);
+              a[1][0] = and_or(wg[j] >> 4, M4, HI);
+              a[1][1] = and_or(wg8[j] >> 4, M4, HI);
+              a[1][2] = and_or(wg[j] >> 12, M4, HI);
+              a[1][3] = and_or(wg8[j] >> 12, M4, HI);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_bf16_16816(cacc[nt], a[0], bfr[nt][j][0][0], bfr[nt][j][0][1]);
+              mma_bf16_16816(cacc[nt], a[1], bfr[nt][j][1][0], bfr[nt][j][1][1]);
+            }
+          }
+          // scales and biases of rows g and g+8 for this group
+          const uint16_t* sm = sb + (m * 2) * kRows * C::KB_PER_CHUNK + C::CW * i;
+          const uint16_t* bm = sm + kRows * C::KB_PER_CHUNK;
+          const float s0 = bf16_to_f32(sm[0]);
+          const float s1 = bf16_to_f32(sm[8 * C::KB_PER_CHUNK]);
+          const float c0 = fmaf(-C::OFFSET, s0, bf16_to_f32(bm[0]));
+          const float c1 = fmaf(-C::OFFSET, s1, bf16_to_f32(bm[8 * C::KB_PER_CHUNK]));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[m][nt][0] = fmaf(s0, cacc[nt][0], fmaf(c0, cx[nt][0], acc[m][nt][0]));
+            acc[m][nt][1] = fmaf(s0, cacc[nt][1], fmaf(c0, cx[nt][1], acc[m][nt][1]));
+            acc[m][nt][2] = fmaf(s1, cacc[nt][2], fmaf(c1, cx[nt][2], acc[m][nt][2]));
+            acc[m][nt][3] = fmaf(s1, cacc[nt][3], fmaf(c1, cx[nt][3], acc[m][nt][3]));
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    ++it;
+    if (++ch == NCH) {
+      finish_unit();
+      ch = 0;
+      ++u;
+      ti = ti_next;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) rows[nt] = rows_next[nt];
+      if (u + 1 < u_end) tile_rows(u + 1, ti_next, rows_next);
+    }
+  };
+
+  const int64_t steps = (u_end - u_begin) * NCH;
+  // Two token sets with wide lanes hold too many live values for two inlined copies of
+  // the step: there the next chunk's activations are moved into place instead.
+  constexpr bool kAlternate = !(NT == 2 && C::LANE_BYTES >= 16);
+  if constexpr (kAlternate) {
+    for (int64_t k = 0; k < steps; k += 2) {
+      step(xa, xb);
+      if (k + 1 < steps) step(xb, xa);
+    }
+  } else {
+    for (int64_t k = 0; k < steps; ++k) {
+      step(xa, xb);
 #pragma unroll
       for (int i = 0; i < C::KB_PER_WARP; ++i)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int j = 0; j < C::WORDS; ++j) xc[i][nt][j] = xn[i][nt][j];
-      if (ch + 1 < NCH)
-        load_x(rows, ch + 1, xn);
-      else if (u + 1 < u_end)
-        load_x(rows_next, 0, xn);
-      const int stage = it % C::STAGES;
-      bool ok = false;
-      if (!*abort_flag) {
-        ok = mbar_wait(&full[stage], (it / C::STAGES) & 1, p.d_status);
-        if (!ok) *abort_flag = 1;
-      }
-      if (ok) {
-        const uint8_t* st = smem + stage * C::STAGE_BYTES;
-        const uint16_t* sb = reinterpret_cast<const uint16_t*>(st + C::CODE_BYTES);
-#pragma unroll
-        for (int i = 0; i < C::KB_PER_WARP; ++i) {
-          const int ikb = warp + kConsumerWarps * i;
-          const int64_t kb = ch * C::KB_PER_CHUNK + ikb;
-          if (kb >= KB_TOTAL) break;
-          // ---- B operand: x values of this lane's codes, permuted to the MMA k order
-          uint32_t bfr[NT][C::WORDS][2][2];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-            for (int j = 0; j < C::WORDS; ++j) {
-              if constexpr (BITS == 4) {
-                const uint4 v = xc[i][nt][j];
-                bfr[nt][j][0][0] = prmt(v.x, v.z, 0x5410);
-                bfr[nt][j][0][1] = prmt(v.x, v.z, 0x7632);
-                bfr[nt][j][1][0] = prmt(v.y, v.w, 0x5410);
-                bfr[nt][j][1][1] = prmt(v.y, v.w, 0x7632);
-              } else {
-                const uint2 v = xc[i][nt][j];
-                bfr[nt][j][0][0] = prmt(v.x, v.y, 0x5410);
-                bfr[nt][j][0][1] = prmt(v.x, v.y, 0x7632);
-                bfr[nt][j][1][0] = bfr[nt][j][0][0];
-                bfr[nt][j][1][1] = bfr[nt][j][0][1];
-              }
-            }
-          }
-          // ---- X = sum of x over the group (all-ones A operand)
-          float cx[NT][4];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-            for (int i2 = 0; i2 < 4; ++i2) cx[nt][i2] = 0.f;
-            const uint32_t ones[4] = {ONES, ONES, ONES, ONES};
-#pragma unroll
-            for (int j = 0; j < C::WORDS; ++j) {
-              mma_bf16_16816(cx[nt], ones, bfr[nt][j][0][0], bfr[nt][j][0][1]);
-              if constexpr (BITS == 4) mma_bf16_16816(cx[nt], ones, bfr[nt][j][1][0], bfr[nt][j][1][1]);
-            }
-          }
-          const int lb = ikb * C::KB_BYTES + t * C::LANE_BYTES;  // lane's byte in the chunk row
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            const uint8_t* cm = st + m * C::BOXES * 2048;
-            uint32_t wg[C::WORDS], wg8[C::WORDS];
-            if constexpr (C::LANE_BYTES == 4) {
-              wg[0] = *reinterpret_cast<const uint32_t*>(cm + swz(g, lb));
-              wg8[0] = *reinterpret_cast<const uint32_t*>(cm + swz(g + 8, lb));
-            } else if constexpr (C::LANE_BYTES == 8) {
-              const uint2 a = *reinterpret_cast<const uint2*>(cm + swz(g, lb));
-              const uint2 b = *reinterpret_cast<const uint2*>(cm + swz(g + 8, lb));
-              wg[0] = a.x; wg[1] = a.y; wg8[0] = b.x; wg8[1] = b.y;
-            } else {
-#pragma unroll
-              for (int q = 0; q < C::LANE_BYTES / 16; ++q) {
-                const uint4 a = *reinterpret_cast<const uint4*>(cm + swz(g, lb + 16 * q));
-                const uint4 b = *reinterpret_cast<const uint4*>(cm + swz(g + 8, lb + 16 * q));
-                wg[4 * q + 0] = a.x; wg[4 * q + 1] = a.y; wg[4 * q + 2] = a.z; wg[4 * q + 3] = a.w;
-                wg8[4 * q + 0] = b.x; wg8[4 * q + 1] = b.y; wg8[4 * q + 2] = b.z; wg8[4 * q + 3] = b.w;
-              }
-            }
-            float cacc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-              for (int i2 = 0; i2 < 4; ++i2) cacc[nt][i2] = 0.f;
-#pragma unroll
-            for (int j = 0; j < C::WORDS; ++j) {
-              uint32_t a[2][4];
-              if constexpr (BITS == 4) {
-                const uint32_t M4 = 0x000F000Fu, MAG = 0x43004300u;
-                a[0][0] = and_or(wg[j], M4, MAG);
-                a[0][1] = and_or(wg8[j], M4, MAG);
-                a[0][2] = and_or(wg[j] >> 4, M4, MAG);
-                a[0][3] = and_or(wg8[j] >> 4, M4, MAG);
-                a[1][0] = and_or(wg[j] >> 8, M4, MAG);
-                a[1][1] = and_or(wg8[j] >> 8, M4, MAG);
-                a[1][2] = and_or(wg[j] >> 12, M4, MAG);
-                a[1][3] = and_or(wg8[j] >> 12, M4, MAG);
-              } else {
-                const uint32_t M4 = 0x000F000Fu, LO = 0x43004300u, HI = 0x45004500u;
-                a[0][0] = and_or(wg[j], M4, LO);
-                a[0][1] = and_or(wg8[j], M4, LO);
-                a[0][2] = and_or(wg[j] >> 8, M4, LO);
-                a[0][3] = and_or(wg8[j] >> 8, M4, LO);
-                a[1][0] = and_or(wg[j] >> 4, M4, HI);
-                a[1][1] = and_or(wg8[j] >> 4, M4, HI);
-                a[1][2] = and_or(wg[j] >> 12, M4, HI);
-                a[1][3] = and_or(wg8[j] >> 12, M4, HI);
-              }
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                mma_bf16_16816(cacc[nt], a[0], bfr[nt][j][0][0], bfr[nt][j][0][1]);
-                mma_bf16_16816(cacc[nt], a[1], bfr[nt][j][1][0], bfr[nt][j][1][1]);
-              }
-            }
-            const uint16_t* sm = sb + (m * 2 + 0) * kRows * C::KB_PER_CHUNK + ikb;
-            const uint16_t* bm = sb + (m * 2 + 1) * kRows * C::KB_PER_CHUNK + ikb;
-            const float s0 = bf16_to_f32(sm[g * C::KB_PER_CHUNK]);
-            const float s1 = bf16_to_f32(sm[(g + 8) * C::KB_PER_CHUNK]);
-            const float c0 = fmaf(-C::OFFSET, s0, bf16_to_f32(bm[g * C::KB_PER_CHUNK]));
-            const float c1 = fmaf(-C::OFFSET, s1, bf16_to_f32(bm[(g + 8) * C::KB_PER_CHUNK]));
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              acc[m][nt][0] = fmaf(s0, cacc[nt][0], fmaf(c0, cx[nt][0], acc[m][nt][0]));
-              acc[m][nt][1] = fmaf(s0, cacc[nt][1], fmaf(c0, cx[nt][1], acc[m][nt][1]));
-              acc[m][nt][2] = fmaf(s1, cacc[nt][2], fmaf(c1, cx[nt][2], acc[m][nt][2]));
-              acc[m][nt][3] = fmaf(s1, cacc[nt][3], fmaf(c1, cx[nt][3], acc[m][nt][3]));
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
-    }
-
-    // ---- hand the partial sums to the epilogue warp (valid token columns only)
-    {
-      const uint32_t ui = static_cast<uint32_t>(u - u_begin), b = ui & 1;
-      if (ui >= 2 && !*abort_flag && !mbar_wait(&red_empty[b], ((ui >> 1) - 1) & 1, p.d_status))
-        *abort_flag = 1;
-      float* ub = red + b * C::RED_SLICE;
-      if (!*abort_flag) {
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            float* r = ub + (((warp * NMAT + m) * NT + nt) * kRows) * 8;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              if (static_cast<uint32_t>(nt * 8 + 2 * t + j) < ti.valid) {
-                r[g * 8 + 2 * t + j] = acc[m][nt][j];
-                r[(g + 8) * 8 + 2 * t + j] = acc[m][nt][2 + j];
-              }
-            }
-          }
-      }
-      mbar_arrive(&red_full[b]);  // release: orders this lane's stores
+          for (int j = 0; j < C::WORDS; ++j) xa[i][nt][j] = xb[i][nt][j];
     }
   }
 }
