@@ -7,7 +7,11 @@
 //   out[t] = sum_k scores[t,k] * y_sorted[inv_order[t*top_k+k]]
 //            + sigmoid(x[t] . w_shared_gate) * shared[t]
 //
-// One CTA per token, 16-byte vectors, fp32 accumulation, one bf16 rounding.
+// Grid: tokens x slices of the hidden dimension (one 16-byte vector per thread), so
+// that a handful of decode tokens still spreads over many SMs.  A CTA stages the
+// token's expert positions and scores in shared memory and issues the loads of up to
+// eight expert rows before it accumulates them, instead of walking a chain of
+// dependent index and row loads.  fp32 accumulation in k order, one bf16 rounding.
 // HBM-bound: per token it reads top_k + 2 rows and the gate vector, writes one row.
 #include "qmoe_common.cuh"
 #include "qmoe_internal.h"
@@ -15,7 +19,9 @@
 namespace qmoe {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
+constexpr int kKChunk = 32;   // expert slots staged in shared memory at a time
+constexpr int kKBatch = 8;    // expert rows loaded before they are accumulated
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -33,19 +39,24 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
     int64_t H, uint16_t* __restrict__ out, int* d_status, ProfSlot* prof) {
   __shared__ float red[kThreads / 32];
   __shared__ float gate_sh;
+  __shared__ uint32_t pos_sh[kKChunk];
+  __shared__ float score_sh[kKChunk];
   const int64_t t = blockIdx.x;
   const int tid = threadIdx.x;
   if (tid == 0) prof_start(prof);
   const int64_t nvec = H / 8;
-  const int64_t R = T * top_k;
+  const int64_t v = static_cast<int64_t>(blockIdx.y) * kThreads + tid;  // this thread's vector
+  const bool live = v < nvec;
+  const uint32_t R = static_cast<uint32_t>(T * top_k);
 
+  // shared-expert gate: sigmoid(x[t] . w_sg), reduced over the whole row by every CTA
   float gate = 1.0f;
   if (shared != nullptr && w_sg != nullptr) {
     float dot = 0.f;
-    for (int64_t v = tid; v < nvec; v += kThreads) {
+    for (int64_t w = tid; w < nvec; w += kThreads) {
       float a[8], b[8];
-      bf16x8_to_f32(reinterpret_cast<const uint4*>(x + t * H)[v], a);
-      bf16x8_to_f32(reinterpret_cast<const uint4*>(w_sg)[v], b);
+      bf16x8_to_f32(reinterpret_cast<const uint4*>(x + t * H)[w], a);
+      bf16x8_to_f32(reinterpret_cast<const uint4*>(w_sg)[w], b);
 #pragma unroll
       for (int i = 0; i < 8; ++i) dot = fmaf(a[i], b[i], dot);
     }
@@ -61,20 +72,41 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
     gate = gate_sh;
   }
 
-  for (int64_t v = tid; v < nvec; v += kThreads) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < top_k; ++k) {
-      const uint32_t pos = inv_order[t * top_k + k];
-      if (pos >= R) {
-        if (v == tid) set_status(d_status, QMOE_DEV_BAD_INDEX);
-        continue;
-      }
-      const float s = scores[t * top_k + k];
-      float yv[8];
-      bf16x8_to_f32(reinterpret_cast<const uint4*>(y_sorted + static_cast<int64_t>(pos) * H)[v], yv);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(s, yv[i], acc[i]);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < top_k; k0 += kKChunk) {
+    const int kn = min(kKChunk, top_k - k0);
+    if (tid < kn) {
+      const uint32_t pos = inv_order[t * top_k + k0 + tid];
+      if (pos >= R && blockIdx.y == 0) set_status(d_status, QMOE_DEV_BAD_INDEX);
+      pos_sh[tid] = pos;
+      score_sh[tid] = scores[t * top_k + k0 + tid];
     }
+    __syncthreads();
+    if (live) {
+      for (int kb = 0; kb < kn; kb += kKBatch) {
+        uint4 yv[kKBatch];
+#pragma unroll
+        for (int j = 0; j < kKBatch; ++j) {
+          yv[j] = make_uint4(0, 0, 0, 0);
+          const uint32_t pos = kb + j < kn ? pos_sh[kb + j] : R;
+          if (pos < R)  // an out-of-range position contributes nothing (status set above)
+            yv[j] = reinterpret_cast<const uint4*>(y_sorted + static_cast<int64_t>(pos) * H)[v];
+        }
+#pragma unroll
+        for (int j = 0; j < kKBatch; ++j) {
+          if (kb + j < kn && pos_sh[kb + j] < R) {
+            const float s = score_sh[kb + j];
+            float yf[8];
+            bf16x8_to_f32(yv[j], yf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(s, yf[i], acc[i]);
+          }
+        }
+      }
+    }
+    __syncthreads();  // before the next chunk overwrites pos_sh / score_sh
+  }
+  if (live) {
     if (shared != nullptr) {
       float sv[8];
       bf16x8_to_f32(reinterpret_cast<const uint4*>(shared + t * H)[v], sv);
@@ -99,9 +131,13 @@ cudaError_t launch_combine(const uint16_t* y_sorted, const uint32_t* inv_order,
                            const uint16_t* w_sg, int64_t T, int top_k, int64_t H, uint16_t* out,
                            int* d_status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
+  if (T > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  const int64_t slices = (H / 8 + kThreads - 1) / kThreads;
+  if (slices > 65535) return cudaErrorInvalidValue;
   LaunchTimer timer("combine", stream);
-  combine_kernel<<<static_cast<unsigned>(T), kThreads, 0, stream>>>(
-      y_sorted, inv_order, scores, shared, x, w_sg, T, top_k, H, out, d_status, timer.slot());
+  const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>(slices));
+  combine_kernel<<<grid, kThreads, 0, stream>>>(y_sorted, inv_order, scores, shared, x, w_sg, T,
+                                                top_k, H, out, d_status, timer.slot());
   count_launch();
   return cudaGetLastError();
 }

@@ -207,19 +207,66 @@ __global__ void __launch_bounds__(kChunk) route_scatter_kernel(RouteDev d) {
   __syncthreads();
   if (threadIdx.x == 0) prof_end(d.prof);
 }
-// R <= 1024: all three phases in one CTA.  Global writes of one phase are read by
-// other threads of the same CTA after __syncthreads.
+// R <= 1024: all three phases in one CTA.
 __global__ void __launch_bounds__(kChunk) route_fused_kernel(RouteDev d) {
-  extern __shared__ uint8_t cnt[];
+  // Shared scratch: per-warp counts [32][E+1] bytes, then the expert bases [E+1].
+  // Every thread keeps its own row's key, x row and stable rank in registers across
+  // the phases, so nothing round-trips through global memory inside the CTA.
+  extern __shared__ uint8_t dyn[];
   __shared__ uint32_t sh[32];
-  if (threadIdx.x == 0) prof_start(d.prof);
-  phase_count(d, 0, cnt);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t nb = d.E + 1;
+  uint8_t* cnt = dyn;
+  uint32_t* base = reinterpret_cast<uint32_t*>(dyn + ((32 * nb + 15) & ~int64_t(15)));
+  if (tid == 0) prof_start(d.prof);
+  for (int64_t i = tid; i < 32 * nb; i += blockDim.x) cnt[i] = 0;
+  const int64_t r = tid;
+  uint32_t key = kNoRow, xrow = 0;
+  if (r < d.R) key = row_key(d, r, &xrow);
   __syncthreads();
-  phase_scan(d, 1, sh);
+  // stable rank: rank inside the warp's equal keys + equal keys of earlier warps
+  const uint32_t mask = __match_any_sync(0xFFFFFFFFu, key);
+  const uint32_t rank = __popc(mask & ((1u << lane) - 1u));
+  if (key != kNoRow && rank == 0) cnt[warp * nb + key] = static_cast<uint8_t>(__popc(mask));
   __syncthreads();
-  phase_scatter(d, 0);
+  uint32_t lrank = rank;
+  if (key != kNoRow)
+    for (int w = 0; w < warp; ++w) lrank += cnt[w * nb + key];
+  // expert totals -> exclusive scan -> bases (shared) and offsets (global)
+  uint32_t carry = 0;
+  for (int64_t e0 = 0; e0 < nb; e0 += blockDim.x) {
+    const int64_t e = e0 + tid;
+    uint32_t tot = 0;
+    if (e < nb)
+      for (int w = 0; w < 32; ++w) tot += cnt[w * nb + e];
+    uint32_t total;
+    const uint32_t off = carry + block_exclusive_scan(tot, sh, &total);
+    if (e < nb) {
+      base[e] = off;
+      d.offsets[e] = off;
+    }
+    carry += total;
+  }
   __syncthreads();
-  if (threadIdx.x == 0) prof_end(d.prof);
+  if (d.tiles != nullptr)
+    write_tiles(base, d.E, d.bm, d.tiles, d.max_tiles, d.num_tiles, d.d_status, sh);
+  // scatter
+  if (r < d.R) {
+    const uint32_t pos = base[key] + lrank;
+    d.order[pos] = static_cast<uint32_t>(r);
+    d.inv_order[r] = pos;
+    if (d.src_row) d.src_row[pos] = xrow;
+    if (key == static_cast<uint32_t>(d.E)) {
+      set_status(d.d_status, QMOE_DEV_BAD_INDEX);
+      if (d.zero_out != nullptr) {
+        const int64_t row = d.zero_by_pos ? static_cast<int64_t>(pos) : r;
+        uint16_t* dst = d.zero_out + row * d.zero_cols;
+        for (int64_t c = 0; c < d.zero_cols; ++c) dst[c] = 0;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) prof_end(d.prof);
 }
 __global__ void __launch_bounds__(kChunk)
     tile_table_kernel(const uint32_t* offsets, int64_t E, int bm, uint32_t* tiles,
@@ -283,17 +330,18 @@ cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream) {
   d.d_status = a.d_status;
   const int64_t nchunks = (R + kChunk - 1) / kChunk;
   const size_t cnt_bytes = static_cast<size_t>(32 * (a.E + 1));
+  const size_t fused_bytes = ((cnt_bytes + 15) & ~size_t(15)) + 4 * static_cast<size_t>(a.E + 1);
   if (cnt_bytes > 200 * 1024) return cudaErrorInvalidValue;  // E above ~6400 experts
-  if (cnt_bytes > 48 * 1024) {
-    cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(cnt_bytes));
+  if (cnt_bytes > 48 * 1024)
     cudaFuncSetAttribute(route_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(cnt_bytes));
-  }
-  if (nchunks <= 1) {
+  if (nchunks <= 1 && fused_bytes <= 220 * 1024) {
+    if (fused_bytes > 48 * 1024)
+      cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(fused_bytes));
     LaunchTimer timer("route", stream);
     d.prof = timer.slot();
-    route_fused_kernel<<<1, kChunk, cnt_bytes, stream>>>(d);
+    route_fused_kernel<<<1, kChunk, fused_bytes, stream>>>(d);
     count_launch();
   } else {
     {
