@@ -13,9 +13,10 @@
 // for the SwitchGLU, or two adjacent 128-channel blocks of one weight stack.  Warps:
 //   0-3   epilogue: tcgen05.ld of the finished accumulators (one TMEM lane = one row),
 //         silu*mul, bf16 stores to the routed rows;
-//   4     producer: 2-D TMA of the activation tile (128 rows x 64 k, 128B-swizzled),
-//         the packed code tiles (128 rows x 64 codes per stack) and, every 8 groups,
-//         the scales and biases;
+//   4     producer: 2-D TMA of the activation tile (128 rows x 64 k, 128B-swizzled)
+//         for every k stage; every 128/(8*bits) k stages, 128 bytes of packed codes of
+//         each of the 128 rows per stack (128B-swizzled, own two-slot ring); every 8
+//         groups, the scales and biases;
 //   5     MMA issuer: owns 512 TMEM columns (two double-buffered unit accumulators),
 //         one thread issues tcgen05.mma kind::f16 (M=128, N=128, K=16) and commits to
 //         mbarriers;
@@ -38,7 +39,6 @@ namespace {
 constexpr int kBM = 128;            // rows per tile = TMEM lanes
 constexpr int kBN = 128;            // output channels per accumulator
 constexpr int kBK = 64;             // k per stage: one 128-byte swizzle atom of bf16
-constexpr int kS2 = 2;              // dequantised-weight ring
 constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps = 8;
 constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;  // 448
 constexpr int kTmemCols = 512;      // 2 buffers x 2 accumulators x 128 columns
@@ -46,16 +46,23 @@ constexpr int kSbGroups = 8;        // groups per scale/bias TMA box (16 bytes o
 
 template <int BITS>
 struct TcCfg {
-  static constexpr int S1 = BITS == 4 ? 5 : 4;                   // activation + packed-code ring
+#ifndef QMOE_TC_S1_4BIT
+#define QMOE_TC_S1_4BIT 5
+#define QMOE_TC_S2_4BIT 2
+#endif
+  static constexpr int S1 = BITS == 4 ? QMOE_TC_S1_4BIT : 4;     // activation + packed-code ring
+  static constexpr int S2 = BITS == 4 ? QMOE_TC_S2_4BIT : 2;     // dequantised-weight ring
   static constexpr int A_BYTES = kBM * kBK * 2;                  // 16 KB
   static constexpr int P_ROW = kBK * BITS / 8;                   // packed bytes per row per stage
-  static constexpr int P_BYTES = 2 * kBM * P_ROW;                // two stacks
+  static constexpr int PK = 128 / P_ROW;                         // stages per packed-code load
+  static constexpr int SP = 2;                                   // packed-code ring
+  static constexpr int P_SLOT = 2 * kBM * 128;                   // two stacks, 128 B per row
   static constexpr int B_BYTES = 2 * kBN * kBK * 2;              // two stacks, bf16
   static constexpr int SB_BYTES = 2 * 2 * kBM * kSbGroups * 2;   // [stack][s|b][row][8]
   static constexpr int OFF_A = 0;
   static constexpr int OFF_P = OFF_A + S1 * A_BYTES;
-  static constexpr int OFF_B = OFF_P + S1 * P_BYTES;
-  static constexpr int OFF_SB = OFF_B + kS2 * B_BYTES;
+  static constexpr int OFF_B = OFF_P + SP * P_SLOT;
+  static constexpr int OFF_SB = OFF_B + S2 * B_BYTES;
   static constexpr int OFF_BAR = OFF_SB + 2 * SB_BYTES;
   static constexpr int SMEM = OFF_BAR + 256;
   static_assert(SMEM + 1024 <= 227 * 1024, "shared memory budget");
@@ -64,7 +71,7 @@ struct TcCfg {
 
 struct alignas(64) TcParams {
   CUtensorMap tm_a;        // activation rows [x_rows, K] bf16, box {64, 128}, 128B swizzle
-  CUtensorMap tm_w[2];     // packed codes [E*N, K*bits/32] u32, box {64*bits/32, 128}
+  CUtensorMap tm_w[2];     // packed codes [E*N, K*bits/32] u32, box {32, 128}, 128B swizzle
   CUtensorMap tm_sb[2][2]; // scales / biases [E*N, K/group] bf16, box {8, 128}
   uint16_t* y;
   const uint32_t* dst_row;
@@ -196,6 +203,7 @@ template <int BITS, int GS>
 __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<BITS>;
   constexpr int kS1 = C::S1;
+  constexpr int kS2 = C::S2;
   // stages covered by one scale/bias box of kSbGroups groups
   constexpr int KS_SB = kSbGroups * GS / kBK;
   static_assert(KS_SB >= 1 && (kSbGroups * GS) % kBK == 0, "group size");
@@ -212,14 +220,20 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
   uint64_t* tfull = empty_sb + 2;         // [2] MMA commit: accumulator ready
   uint64_t* tempty = tfull + 2;           // [2] epilogue warps: accumulator drained
   uint64_t* drain = tempty + 2;           // [1] final MMA commit on the abort path
-  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* fullP = drain + 1;            // [SP] TMA tx (packed codes)
+  uint64_t* emptyP = fullP + C::SP;       // [SP] dequant warps
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(emptyP + C::SP);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kS1; ++s) {
       mbar_init(&full1[s], 1);
-      mbar_init(&empty1[s], 1 + kDqWarps);
+      mbar_init(&empty1[s], 1);
+    }
+    for (int s = 0; s < C::SP; ++s) {
+      mbar_init(&fullP[s], 1);
+      mbar_init(&emptyP[s], kDqWarps);
     }
     for (int s = 0; s < kS2; ++s) {
       mbar_init(&full2[s], kDqWarps);
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_a);
-      uint32_t it = 0, sbit = 0;
+      uint32_t it = 0, sbit = 0, pbit = 0;
       bool ab = false;
       for (int64_t u = u_begin; u < u_end && !ab; u += u_step) {
         const Tile tl = tc_tile(p, u / NBLK);
@@ -282,16 +296,23 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
                             static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
             ++sbit;
           }
+          if (ks % C::PK == 0) {
+            // packed codes of the next PK stages: 128 bytes of each row, 128B-swizzled
+            const uint32_t ps = pbit % C::SP;
+            if (!mbar_wait(&emptyP[ps], ((pbit / C::SP) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+            mbar_arrive_expect_tx(&fullP[ps], C::P_SLOT);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+              tma_load_2d(smem + C::OFF_P + ps * C::P_SLOT + m * kBM * 128, &p.tm_w[m], &fullP[ps],
+                          static_cast<int32_t>(ks * kBK * BITS / 32),
+                          static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
+            ++pbit;
+          }
           const uint32_t s1 = it % kS1;
           if (!mbar_wait(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
-          mbar_arrive_expect_tx(&full1[s1], C::A_BYTES + C::P_BYTES);
+          mbar_arrive_expect_tx(&full1[s1], C::A_BYTES);
           tma_load_2d(smem + C::OFF_A + s1 * C::A_BYTES, &p.tm_a, &full1[s1],
                       static_cast<int32_t>(ks * kBK), static_cast<int32_t>(tl.row_start));
-#pragma unroll
-          for (int m = 0; m < 2; ++m)
-            tma_load_2d(smem + C::OFF_P + s1 * C::P_BYTES + m * kBM * C::P_ROW, &p.tm_w[m],
-                        &full1[s1], static_cast<int32_t>(ks * kBK * BITS / 32),
-                        static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
           ++it;
         }
       }
@@ -301,6 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         for (uint32_t k = first; k < it; ++k) mbar_wait(&full1[k % kS1], (k / kS1) & 1, nullptr);
         const uint32_t sfirst = sbit > 2u ? sbit - 2 : 0u;
         for (uint32_t k = sfirst; k < sbit; ++k) mbar_wait(&full_sb[k & 1], (k >> 1) & 1, nullptr);
+        const uint32_t pfirst = pbit > static_cast<uint32_t>(C::SP) ? pbit - C::SP : 0u;
+        for (uint32_t k = pfirst; k < pbit; ++k)
+          mbar_wait(&fullP[k % C::SP], (k / C::SP) & 1, nullptr);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -354,16 +378,18 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     // packed tile and write distinct swizzled 16-byte chunks (no bank conflicts).
     const int dq = threadIdx.x - kDqWarp0 * 32;  // 0..255
     constexpr int HALF = C::P_ROW / 2;           // packed bytes per half-row: 16 or 32
-    uint32_t it = 0, sbit = 0;
+    uint32_t it = 0, sbit = 0, pbit = 0;
     for (int64_t u = u_begin; u < u_end; u += u_step) {
       for (int64_t ks = 0; ks < KS; ++ks, ++it) {
         if (*abort_flag) break;
         const uint32_t e = sbit & 1;
         if (ks % KS_SB == 0 &&
             !mbar_wait(&full_sb[e], (sbit >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
-        const uint32_t s1 = it % kS1, s2 = it % kS2;
-        if (!mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) ||
-            !mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+        const uint32_t ps = pbit % C::SP, s2 = it % kS2;
+        if (ks % C::PK == 0 &&
+            !mbar_wait(&fullP[ps], (pbit / C::SP) & 1, p.d_status)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+        const int pj = static_cast<int>(ks % C::PK);  // stage inside the packed rows
         const int gin = static_cast<int>((ks * kBK / GS) % kSbGroups);
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
@@ -372,12 +398,14 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
           const uint16_t* sbp = reinterpret_cast<const uint16_t*>(smem + C::OFF_SB + e * C::SB_BYTES) +
                                 ((m * 2) * kBM + row) * kSbGroups;
           const uint16_t* bbp = sbp + kBM * kSbGroups;
-          const uint8_t* prow = smem + C::OFF_P + s1 * C::P_BYTES + (m * kBM + row) * C::P_ROW + half * HALF;
+          // packed row: 128 bytes, 16-byte chunk c stored at chunk c ^ (row & 7)
+          const uint8_t* prow = smem + C::OFF_P + ps * C::P_SLOT + (m * kBM + row) * 128;
+          const int pc = (pj * C::P_ROW + half * HALF) / 16;  // first chunk of this half-row
           uint8_t* brow = smem + C::OFF_B + s2 * C::B_BYTES + (m * kBN + row) * (kBK * 2);
           // codes 32*half .. 32*half+31 of this row's 64
           const int gj = gin + (GS == 32 ? half : 0);
           if constexpr (BITS == 4) {
-            const uint4 pw = *reinterpret_cast<const uint4*>(prow);
+            const uint4 pw = *reinterpret_cast<const uint4*>(prow + ((pc ^ (row & 7)) << 4));
             const uint32_t w[4] = {pw.x, pw.y, pw.z, pw.w};
             const uint16_t sv = sbp[gj], bv = bbp[gj];
             const __nv_bfloat162 s2v = __halves2bfloat162(__ushort_as_bfloat16(sv), __ushort_as_bfloat16(sv));
@@ -388,8 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
               *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = dequant_word4(w[j], s2v, b2v);
             }
           } else {
-            const uint4 pa = *reinterpret_cast<const uint4*>(prow);
-            const uint4 pb = *reinterpret_cast<const uint4*>(prow + 16);
+            const uint4 pa = *reinterpret_cast<const uint4*>(prow + ((pc ^ (row & 7)) << 4));
+            const uint4 pb = *reinterpret_cast<const uint4*>(prow + (((pc + 1) ^ (row & 7)) << 4));
             const uint32_t w[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
             const float sv = bf16_to_f32(sbp[gj]), bv = bf16_to_f32(bbp[gj]);
 #pragma unroll
@@ -403,11 +431,13 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         }
         fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
         __syncwarp();
+        const bool p_done = ks % C::PK == C::PK - 1 || ks == KS - 1;
         if (lane == 0) {
           mbar_arrive(&full2[s2]);
-          mbar_arrive(&empty1[s1]);
+          if (p_done) mbar_arrive(&emptyP[ps]);
           if (ks % KS_SB == KS_SB - 1 || ks == KS - 1) mbar_arrive(&empty_sb[e]);
         }
+        if (p_done) ++pbit;
         if (ks % KS_SB == KS_SB - 1 || ks == KS - 1) ++sbit;
       }
       if (*abort_flag) break;
@@ -523,8 +553,9 @@ cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream) {
   const int64_t gpr = a.K / a.group;
   for (int m = 0; m < 2; ++m) {
     const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
-    e = make_tmap_2d_u32(&prm.tm_w[m], wm.codes, words, a.E * a.N, kBK * a.bits / 32, kBM,
-                         /*swizzle128=*/false);
+    // 128 bytes of each row (several k stages) per copy, 128B-swizzled
+    e = make_tmap_2d_u32(&prm.tm_w[m], wm.codes, words, a.E * a.N, 32, kBM,
+                         /*swizzle128=*/true);
     if (e != cudaSuccess) return e;
     e = make_tmap_2d_bf16(&prm.tm_sb[m][0], wm.scales, gpr, a.E * a.N, kSbGroups, kBM, false);
     if (e != cudaSuccess) return e;
