@@ -13,10 +13,13 @@ step touches / step time.  Weights (3.6 GB) are far larger than L2, and fresh
 routing per layer keeps each layer's experts cold.
 
 Printed on rank 0 as one JSON line, with: isolated decode layers at M=1 and M=4;
-the prefill MoE layer (T=4096, Zipf-skewed routing); the roofline of the dominant
-kernel (timed live with CUDA events around each launch); an end-to-end number with
-host buffers; SM clocks sampled through NVML during the timed region; and the CPU
-oracle timed on a bounded sample (rank 0, N=1).
+the prefill MoE layer at T = 512 ... 16384 (Zipf-skewed routing); the dense small-M
+decoder-block qmm forward (1..16 rows, 4- and 8-bit); the full MoE block with a
+shared expert and the combine (4-bit g64 and 8-bit g128); the roofline of the
+dominant kernel (its launches timed live by the kernels' own device timers inside
+the CUDA graph); an end-to-end number with host buffers; SM clocks sampled through
+NVML during the timed region; and the CPU oracle timed on a bounded sample (rank 0,
+N=1).
 
 ``--impl reference`` times the CPU oracle itself (the reference arm of this
 repository) on the same metric.  Under torchrun each rank runs an independent
@@ -173,6 +176,14 @@ def sum_over_ranks(value: float, ws: int) -> float:
     return float(t.item())
 
 
+def job_gbs(my_bytes: float, my_ms: float, ws: int):
+    """Whole-job throughput of independent replicas: the bytes every rank processed
+    over the slowest rank's time.  Returns (GB/s, max ms)."""
+    ms_max = max_over_ranks(my_ms, ws)
+    total = sum_over_ranks(my_bytes, ws)
+    return total / (ms_max * 1e-3) / 1e9, ms_max
+
+
 def barrier(ws):
     if ws > 1:
         import torch.distributed as dist
@@ -300,9 +311,132 @@ def run_prefill(q, token_counts, dev, peaks, reps=5):
         dn_ms = split["tc"] or split["qmv"]
         glu_tf = T * TOP_K * 4 * 2048 * 512 / (glu_ms * 1e-3) / 1e12 if glu_ms else None
         dn_tf = T * TOP_K * 2 * 2048 * 512 / (dn_ms * 1e-3) / 1e12 if dn_ms else None
+        # bytes the layer must move at least: touched experts' weights, the activations
+        # read and the expert outputs written (x once, x_s and y_sorted, h both ways)
+        touched = len(np.unique(d["idx"]))
+        R = T * TOP_K
+        moved = touched * (2 * matrix_bytes(512, 2048) + matrix_bytes(2048, 512)) + \
+            T * 2048 * 2 + R * 512 * 4 + R * 2048 * 2
+        gbs = moved / (t * 1e-3) / 1e9
+        hbm_peak = peaks["hbm_gbs"] if peaks else 6650.0
         out[f"T{T}"] = {"ms": t, "tflops": tf, "frac_bf16_peak": tf / bf16_peak,
+                        "bytes_moved": moved, "gbs": gbs, "frac_hbm": gbs / hbm_peak,
+                        "touched_experts": touched,
                         "kernel_ms": split, "upgate_tflops": glu_tf, "down_tflops": dn_tf}
         del Wp, d
+    return out
+
+
+def _graph_time(fn, reps=8):
+    """Device time of one replay of a CUDA graph of fn (ms): 3 warm replays, then reps
+    replays between CUDA events on the current stream."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / reps
+    del g
+    return t
+
+
+def run_dense(q, dev, peaks, layers=36, n_sets=8):
+    """Dense small-M quantised matmuls over decoder-block shapes (hidden 2560, q 4096,
+    kv 1024, intermediate 9728): a forward of 36 layers of q/k/v/o/gate/up/down qmm,
+    cycling over 8 weight sets so the weights (>= 454 MB) stream from HBM, for 1..16
+    rows, 4-bit and 8-bit group 64.  Weights W = N(0,1)/sqrt(K) bf16, quantised by
+    qmoe_quantize.  Reports forward time and weight GB/s against the HBM peak."""
+    import torch
+    from inputs import dense_projections
+    proj = dense_projections()
+    hbm = peaks["hbm_gbs"] if peaks else 6650.0
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3)
+    out = {}
+    for bits in (4, 8):
+        sets = []
+        for _ in range(n_sets):
+            layer = []
+            for _, N, K in proj:
+                w = (torch.randn(N, K, generator=gen, device=dev) / K ** 0.5).to(torch.bfloat16)
+                layer.append(q.qmoe_quantize(w, GROUP, bits))
+                del w
+            sets.append(layer)
+        layer_bytes = sum(matrix_bytes(N, K, GROUP, bits) for _, N, K in proj)
+        rows = {}
+        for M in (1, 2, 3, 4, 5, 6, 7, 8, 10, 12, 16):
+            xs = {K: torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)
+                  for K in sorted({k for _, _, k in proj})}
+            ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _, N, _ in proj]
+
+            def fwd():
+                for l in range(layers):
+                    ws = sets[l % n_sets]
+                    for i, (_, N, K) in enumerate(proj):
+                        q.qmoe_qmm(xs[K], *ws[i], GROUP, bits, out=ys[i])
+
+            t = _graph_time(fwd)
+            gbs = layers * layer_bytes / (t * 1e-3) / 1e9
+            rows[f"M{M}"] = {"ms": t, "weight_gbs": gbs, "frac_hbm": gbs / hbm}
+        out[f"{bits}bit_g{GROUP}"] = {"bytes_per_forward": layers * layer_bytes, "rows": rows}
+        del sets
+    return out
+
+
+def run_block(q, dev, peaks):
+    """Full MoE block: the prefill routing at T in {128, 331, 2048, 4096}, expert-sorted
+    routed SwitchGLU, a shared SwiGLU expert (intermediate 512, same quantisation), and
+    the one-pass combine with the sigmoid-gated shared output; 4-bit group 64 and 8-bit
+    group 128.  Reports block time, TFLOP/s and the weight bytes touched per second."""
+    import torch
+    from gpu_util import dev_bf16, dev_f32, dev_u32, qweight
+    from inputs import prefill_layer
+    hbm = peaks["hbm_gbs"] if peaks else 6650.0
+    bf16_peak = peaks["bf16_tflops"] if peaks else 1590.0
+    out = {}
+    for bits, group in ((4, 64), (8, 128)):
+        e_bytes = 2 * matrix_bytes(512, 2048, group, bits) + matrix_bytes(2048, 512, group, bits)
+        res = {}
+        for T in (128, 331, 2048, 4096):
+            d = prefill_layer(0, T, group=group, bits=bits, shared=True)
+            W = [qweight(*d[k], group, bits) for k in ("up", "gate", "down")]
+            S = [qweight(*d[k], group, bits) for k in ("sh_up", "sh_gate", "sh_down")]
+            xd, ids, sc, wsg = dev_bf16(d["x"]), dev_u32(d["idx"]), dev_f32(d["scores"]), dev_bf16(d["w_sg"])
+            zeros = torch.zeros((T, 1), dtype=torch.int32, device=dev)
+            ws1 = torch.empty(q.qmoe_switch_glu_workspace_size(T, TOP_K, *W), dtype=torch.uint8, device=dev)
+            ws2 = torch.empty(q.qmoe_switch_glu_workspace_size(T, 1, *S), dtype=torch.uint8, device=dev)
+            ys = torch.empty((T * TOP_K, 2048), dtype=torch.bfloat16, device=dev)
+            inv = torch.empty(T * TOP_K, dtype=torch.int32, device=dev)
+            sh = torch.empty((T, 1, 2048), dtype=torch.bfloat16, device=dev)
+            ob = torch.empty((T, 2048), dtype=torch.bfloat16, device=dev)
+
+            def blk():
+                q.qmoe_switch_glu(xd, ids, *W, mode=1, out=ys, inv_order=inv, workspace=ws1)
+                q.qmoe_switch_glu(xd, zeros, *S, mode=0, out=sh, workspace=ws2)
+                q.qmoe_moe_combine(ys, inv, sc, sh.view(T, 2048), xd, wsg, out=ob)
+
+            t = _graph_time(blk)
+            touched = len(np.unique(d["idx"]))
+            flop = (T * TOP_K + T) * PREFILL_FLOP_PER_ROW
+            wbytes = (touched + 1) * e_bytes
+            res[f"T{T}"] = {"ms": t, "tflops": flop / (t * 1e-3) / 1e12,
+                            "frac_bf16_peak": flop / (t * 1e-3) / 1e12 / bf16_peak,
+                            "touched_experts": touched,
+                            "weight_gbs": wbytes / (t * 1e-3) / 1e9,
+                            "frac_hbm_weights": wbytes / (t * 1e-3) / 1e9 / hbm}
+            del W, S, d
+        out[f"{bits}bit_g{group}"] = res
     return out
 
 
@@ -319,8 +453,12 @@ def main():
                    help="number of experts (smaller for profiling captures)")
     p.add_argument("--prefill-only", type=int, default=0, metavar="T",
                    help="only time the prefill MoE layer at T tokens (profiling captures)")
-    p.add_argument("--prefill-tokens", default="4096,16384",
+    p.add_argument("--prefill-tokens", default="512,713,1024,2048,4123,8192,16384",
                    help="comma-separated token counts of the prefill measurement")
+    p.add_argument("--no-dense", action="store_true",
+                   help="skip the dense small-M decoder-block qmm forward")
+    p.add_argument("--no-block", action="store_true",
+                   help="skip the MoE block with shared expert and combine")
     args = p.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, ws, local = dist_setup(args.gpus)
@@ -408,13 +546,11 @@ def main():
     barrier(ws)
     ms = e0.elapsed_time(e1)
     launches = launches_per_step * args.steps
-    ms_max = max_over_ranks(ms, ws)
     my_bytes = sum(step_bytes(s) for s in range(args.warmup, args.warmup + args.steps))
-    total_bytes = sum_over_ranks(my_bytes, ws)
-    value = total_bytes / (ms_max * 1e-3) / 1e9
+    value, ms_max = job_gbs(my_bytes, ms, ws)
     ms_per_step = ms_max / args.steps
 
-    # instrumented graph: CUDA events captured around every kernel of the step
+    # instrumented graph: the kernels' device timers around every launch of the step
     slots = torch.zeros(16 * 4 * LAYERS * 4, dtype=torch.uint8, device=dev)
     q.qmoe_timing_enable(slots)
     g_timed, _ = capture()
@@ -472,8 +608,8 @@ def main():
         e2e_step(s)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
-    e2e = {"value": total_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+    e2e_gbs, _ = job_gbs(my_bytes, e0.elapsed_time(e1), ws)
+    e2e = {"value": e2e_gbs, "unit": "GB/s",
            "h2d_bytes_per_step": M_CHAIN * H * 2 + LAYERS * (idx_cur[0].numel() + sc_cur[0].numel()) * 4,
            "d2h_bytes_per_step": M_CHAIN * H * 2}
 
@@ -531,6 +667,9 @@ def main():
         prefill = run_prefill(q, [int(t) for t in args.prefill_tokens.split(",") if t], dev,
                               peaks)
 
+    dense = run_dense(q, dev, peaks) if not args.no_dense else None
+    block = run_block(q, dev, peaks) if not args.no_block else None
+
     # CPU oracle on a bounded sample (rank 0, N = 1)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu and args.experts == E:
@@ -552,7 +691,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(CONFIG, experts=args.experts), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches,
-            "decode_isolated": isolated, "prefill": prefill,
+            "decode_isolated": isolated, "prefill": prefill, "dense_qmm": dense,
+            "moe_block": block,
             "hbm_frac_of_measured": value / hbm_peak,
         }
         print(json.dumps(line), flush=True)

@@ -58,22 +58,23 @@ int64_t max_tiles_for(int64_t R, int64_t E, int bm) {
 
 constexpr int kTcBm = 128;
 
-// Which kernel serves a gathered matmul of R routed rows over E experts.
+// Which kernel serves a gathered matmul of R routed rows over E experts.  The tile
+// tables are built on the device, so the host plans from the most rows one expert can
+// receive (`max_rows`), not from an average: with skewed routing one expert may take
+// most rows even when the average is a few.  Up to 16 rows per expert the streaming
+// kernel (weights read once per tile of 8 or 16 rows) wins; beyond that one 128-row
+// tensor-core tile costs less than the streamed tiles it replaces.
 struct Plan {
   bool tc;
   int bm;
 };
-Plan plan_for(int64_t R, int64_t E, const GemmArgs& probe) {
+Plan plan_for(int64_t R, int64_t E, int64_t max_rows, bool tc_ok) {
+  const Kernel k = forced_kernel();
   const int64_t touched = std::max<int64_t>(1, std::min(E, R));
-  const int64_t avg_rows = R / touched;
-  Kernel k = forced_kernel();
-  bool tc = false;
-  if (k == Kernel::Tc)
-    tc = qmm_tc_supported(probe);
-  else if (k == Kernel::Auto)
-    tc = qmm_tc_supported(probe) && avg_rows >= 32;
-  if (tc) return {true, kTcBm};
-  return {false, avg_rows > 8 ? 16 : 8};
+  const Plan stream{false, R / touched > 8 ? 16 : 8};
+  if (!tc_ok || k == Kernel::Qmv) return stream;
+  if (k == Kernel::Tc || max_rows > 16) return {true, kTcBm};
+  return stream;
 }
 
 struct RouteBufs {
@@ -177,11 +178,13 @@ int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, const qmoe_bf
   a.y = y;
   a.dense_rows = M;
   a.d_status = d_status;
-  const Plan pl = plan_for(M, 1, a);
-  a.bm = pl.bm;
-  a.max_tiles = (M + pl.bm - 1) / pl.bm;
+  // one weight matrix: tensor cores from 32 rows, else the streaming kernel
+  const Kernel k = forced_kernel();
+  const bool tc = qmm_tc_supported(a) && (k == Kernel::Tc || (k == Kernel::Auto && M >= 32));
+  a.bm = tc ? kTcBm : (M > 8 ? 16 : 8);
+  a.max_tiles = (M + a.bm - 1) / a.bm;
   auto s = static_cast<cudaStream_t>(stream);
-  return cuda_status(pl.tc ? launch_qmm_tc(a, s) : launch_qmv(a, s));
+  return cuda_status(tc ? launch_qmm_tc(a, s) : launch_qmv(a, s));
 }
 
 size_t qmoe_gather_qmm_workspace_size(int64_t B, int64_t M, int64_t E, int64_t N, int64_t K) {
@@ -227,7 +230,9 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   a.tiles = rb.tiles;
   a.num_tiles = rb.num_tiles;
   a.d_status = d_status;
-  const Plan pl = plan_for(R, E, a);
+  // Any expert may receive every routed row; below one 128-row tile the streaming
+  // kernel serves every expert.
+  const Plan pl = plan_for(R, E, R > kTcBm ? R : 16, qmm_tc_supported(a));
   a.bm = pl.bm;
   a.max_tiles = max_tiles_for(R, E, pl.bm);
 
@@ -251,16 +256,14 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   ra.zero_by_pos = false;
   ra.d_status = d_status;
   auto s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_route(ra, rb.route_ws, s);
-  if (e != cudaSuccess) return QMOE_ERR_CUDA;
+  if (launch_route(ra, rb.route_ws, s) != cudaSuccess) return QMOE_ERR_CUDA;
   if (pl.tc) {
-    e = launch_gather_rows(x, rb.src_row, R, K, x_sorted, s);
-    if (e != cudaSuccess) return QMOE_ERR_CUDA;
-    a.x = x_sorted;
+    if (launch_gather_rows(x, rb.src_row, R, K, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
+    a.x = x_sorted;  // 128-row tiles over the expert-ordered rows
     a.src_row = nullptr;
     return cuda_status(launch_qmm_tc(a, s));
   }
-  a.x = x;
+  a.x = x;  // the streaming kernel reads x through src_row
   a.src_row = rb.src_row;
   return cuda_status(launch_qmv(a, s));
 }
@@ -367,8 +370,9 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   dn.tiles = rb.tiles;
   dn.num_tiles = rb.num_tiles;
   dn.d_status = d_status;
-  Plan pl = plan_for(R, E, ug);
-  if (pl.tc && !qmm_tc_supported(dn)) pl = Plan{false, pl.bm > 8 ? 16 : 8};
+  // With distinct experts per token one expert receives at most T rows.  The bound only
+  // picks the plan: any routing is served correctly by either kernel.
+  const Plan pl = plan_for(R, E, T, qmm_tc_supported(ug) && qmm_tc_supported(dn));
   ug.bm = dn.bm = pl.bm;
   ug.max_tiles = dn.max_tiles = max_tiles_for(R, E, pl.bm);
 

@@ -80,6 +80,10 @@ struct alignas(64) TcParams {
   int64_t dense_rows;
   int64_t N, K;
   int pair;                // 1: one stack, the two accumulators are adjacent channel blocks
+  int sb_groups;           // > 0: a row has fewer than 8 groups; the unit's scales and
+                           // biases ([128 rows][sb_groups] each) come by 1-D bulk copies
+  const uint16_t* scales[2];
+  const uint16_t* biases[2];
   int* d_status;
   ProfSlot* prof;
 };
@@ -199,14 +203,14 @@ __device__ __forceinline__ uint2 dequant_word8(uint32_t w, float s, float b) {
   return make_uint2(bf16x2_of(v[0], v[1]), bf16x2_of(v[2], v[3]));
 }
 
-template <int BITS, int GS>
+template <int BITS, int GS, bool SB_WHOLE>
 __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<BITS>;
   constexpr int kS1 = C::S1;
   constexpr int kS2 = C::S2;
   // stages covered by one scale/bias box of kSbGroups groups
-  constexpr int KS_SB = kSbGroups * GS / kBK;
-  static_assert(KS_SB >= 1 && (kSbGroups * GS) % kBK == 0, "group size");
+  constexpr int KS_SB_BOX = kSbGroups * GS / kBK;
+  static_assert(KS_SB_BOX >= 1 && (kSbGroups * GS) % kBK == 0, "group size");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -260,6 +264,14 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
   const uint32_t tmem_base = *tmem_base_sh;
 
   const int64_t KS = p.K / kBK;  // k stages per unit
+  // Scale/bias window: one box of 8 groups (KS_SB_BOX stages), or the whole row when it
+  // has fewer groups.  Only compile-time divisors appear in the per-stage tests.
+  constexpr bool sb_whole = SB_WHOLE;  // p.sb_groups > 0
+  const int sb_stride = sb_whole ? p.sb_groups : kSbGroups;  // groups per smem row
+  auto sb_first = [&](int64_t ks) { return sb_whole ? ks == 0 : ks % KS_SB_BOX == 0; };
+  auto sb_last = [&](int64_t ks) {
+    return ks == KS - 1 || (!sb_whole && ks % KS_SB_BOX == KS_SB_BOX - 1);
+  };
   const int unit_n = p.pair ? 2 * kBN : kBN;
   const int64_t NBLK = (p.N + unit_n - 1) / unit_n;
   const int64_t ntiles = p.dense_rows > 0 ? (p.dense_rows + kBM - 1) / kBM : *p.num_tiles;
@@ -282,18 +294,32 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         const int64_t wrow = static_cast<int64_t>(tl.expert) * p.N + n0;
         for (int64_t ks = 0; ks < KS; ++ks) {
           if (*abort_flag) { ab = true; break; }
-          if (ks % KS_SB == 0) {
+          if (sb_first(ks)) {
             const uint32_t e = sbit & 1;
             if (!mbar_wait(&empty_sb[e], ((sbit >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
-            mbar_arrive_expect_tx(&full_sb[e], C::SB_BYTES);
-            const int32_t gx = static_cast<int32_t>(ks * kBK / GS);
+            if constexpr (SB_WHOLE) {
+              // rows wrow.. of one stack are contiguous: [128 rows][sb_groups] per array
+              const uint32_t bytes = kBM * p.sb_groups * 2;
+              mbar_arrive_expect_tx(&full_sb[e], 4 * bytes);
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+              for (int m = 0; m < 2; ++m) {
+                const int64_t r0 = wrow + (p.pair ? kBN * m : 0);
 #pragma unroll
-              for (int arr = 0; arr < 2; ++arr)
-                tma_load_2d(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
-                            &p.tm_sb[m][arr], &full_sb[e], gx,
-                            static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
+                for (int arr = 0; arr < 2; ++arr)
+                  bulk_load(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
+                            (arr ? p.biases[m] : p.scales[m]) + r0 * p.sb_groups, bytes, &full_sb[e]);
+              }
+            } else {
+              mbar_arrive_expect_tx(&full_sb[e], C::SB_BYTES);
+              const int32_t gx = static_cast<int32_t>(ks * kBK / GS);
+#pragma unroll
+              for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int arr = 0; arr < 2; ++arr)
+                  tma_load_2d(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
+                              &p.tm_sb[m][arr], &full_sb[e], gx,
+                              static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
+            }
             ++sbit;
           }
           if (ks % C::PK == 0) {
@@ -383,20 +409,21 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
       for (int64_t ks = 0; ks < KS; ++ks, ++it) {
         if (*abort_flag) break;
         const uint32_t e = sbit & 1;
-        if (ks % KS_SB == 0 &&
+        if (sb_first(ks) &&
             !mbar_wait(&full_sb[e], (sbit >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
         const uint32_t ps = pbit % C::SP, s2 = it % kS2;
         if (ks % C::PK == 0 &&
             !mbar_wait(&fullP[ps], (pbit / C::SP) & 1, p.d_status)) { *abort_flag = 1; break; }
         if (!mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
         const int pj = static_cast<int>(ks % C::PK);  // stage inside the packed rows
-        const int gin = static_cast<int>((ks * kBK / GS) % kSbGroups);
+        const int gin = sb_whole ? static_cast<int>(ks * kBK / GS)
+                                 : static_cast<int>((ks * kBK / GS) % kSbGroups);
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
           const int hr = dq + 256 * rep;          // (stack, row, half)
           const int m = hr / (2 * kBM), row = (hr / 2) % kBM, half = hr & 1;
           const uint16_t* sbp = reinterpret_cast<const uint16_t*>(smem + C::OFF_SB + e * C::SB_BYTES) +
-                                ((m * 2) * kBM + row) * kSbGroups;
+                                (m * 2) * kBM * kSbGroups + row * sb_stride;
           const uint16_t* bbp = sbp + kBM * kSbGroups;
           // packed row: 128 bytes, 16-byte chunk c stored at chunk c ^ (row & 7)
           const uint8_t* prow = smem + C::OFF_P + ps * C::P_SLOT + (m * kBM + row) * 128;
@@ -435,10 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         if (lane == 0) {
           mbar_arrive(&full2[s2]);
           if (p_done) mbar_arrive(&emptyP[ps]);
-          if (ks % KS_SB == KS_SB - 1 || ks == KS - 1) mbar_arrive(&empty_sb[e]);
+          if (sb_last(ks)) mbar_arrive(&empty_sb[e]);
         }
         if (p_done) ++pbit;
-        if (ks % KS_SB == KS_SB - 1 || ks == KS - 1) ++sbit;
+        if (sb_last(ks)) ++sbit;
       }
       if (*abort_flag) break;
     }
@@ -515,10 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
   if (threadIdx.x == 0) prof_end(p.prof);
 }
 
-template <int BITS, int GS>
-cudaError_t launch_tc(TcParams prm, cudaStream_t stream) {
+template <int BITS, int GS, bool SB_WHOLE>
+cudaError_t launch_tc_sb(TcParams prm, cudaStream_t stream) {
   using C = TcCfg<BITS>;
-  auto kern = qmm_tc_kernel<BITS, GS>;
+  auto kern = qmm_tc_kernel<BITS, GS, SB_WHOLE>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -533,12 +560,23 @@ cudaError_t launch_tc(TcParams prm, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int BITS, int GS>
+cudaError_t launch_tc(const TcParams& prm, cudaStream_t stream) {
+  return prm.sb_groups > 0 ? launch_tc_sb<BITS, GS, true>(prm, stream)
+                           : launch_tc_sb<BITS, GS, false>(prm, stream);
+}
+
 }  // namespace
 
 bool qmm_tc_supported(const GemmArgs& a) {
   if (a.bits != 4 && a.bits != 8) return false;
   if (a.K % kBK != 0) return false;
-  if ((a.K / a.group) % kSbGroups != 0) return false;  // scale/bias rows: 16-byte pitch
+  const int64_t gpr = a.K / a.group;
+  // scale/bias rows: a 16-byte pitch for the 2-D boxes, or fewer than 8 groups with
+  // whole units (128 channels of each of two stacks, or 256 of one), so that every
+  // bulk copy of a unit's 128-row blocks stays inside the arrays
+  const int64_t unit_n = a.nmat == 2 ? kBN : 2 * kBN;
+  if (gpr % kSbGroups != 0 && !(gpr < kSbGroups && a.N % unit_n == 0)) return false;
   if (a.x_rows <= 0) return false;
   return true;
 }
@@ -557,11 +595,16 @@ cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream) {
     e = make_tmap_2d_u32(&prm.tm_w[m], wm.codes, words, a.E * a.N, 32, kBM,
                          /*swizzle128=*/true);
     if (e != cudaSuccess) return e;
-    e = make_tmap_2d_bf16(&prm.tm_sb[m][0], wm.scales, gpr, a.E * a.N, kSbGroups, kBM, false);
-    if (e != cudaSuccess) return e;
-    e = make_tmap_2d_bf16(&prm.tm_sb[m][1], wm.biases, gpr, a.E * a.N, kSbGroups, kBM, false);
-    if (e != cudaSuccess) return e;
+    prm.scales[m] = wm.scales;
+    prm.biases[m] = wm.biases;
+    if (gpr % kSbGroups == 0) {
+      e = make_tmap_2d_bf16(&prm.tm_sb[m][0], wm.scales, gpr, a.E * a.N, kSbGroups, kBM, false);
+      if (e != cudaSuccess) return e;
+      e = make_tmap_2d_bf16(&prm.tm_sb[m][1], wm.biases, gpr, a.E * a.N, kSbGroups, kBM, false);
+      if (e != cudaSuccess) return e;
+    }
   }
+  prm.sb_groups = gpr % kSbGroups == 0 ? 0 : static_cast<int>(gpr);
   prm.y = a.y;
   prm.dst_row = a.dst_row;
   prm.tiles = a.tiles;

@@ -54,13 +54,6 @@ namespace qmoe {
 namespace {
 
 constexpr int kRows = 16;             // output channels per unit (MMA M)
-#ifndef QMOE_QMV_PREFETCH_AHEAD
-#define QMOE_QMV_PREFETCH_AHEAD 8
-#endif
-// Chunks the producer prefetches into L2 beyond the one it loads into shared memory.
-// The shared-memory ring alone holds too few bytes in flight while the consumers
-// compute on their stages; the prefetches keep DRAM busy further ahead.
-constexpr int kPrefetchAhead = QMOE_QMV_PREFETCH_AHEAD;
 constexpr int kSmemBudget = 225 * 1024;
 
 // Consumer warps: 8.  With the producer and epilogue warps that is 10 warps (three
@@ -205,37 +198,6 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
         }
       }
     }
-    // L2 prefetch of chunk position `lin` of this CTA's (unit, chunk) sequence (lane 0).
-    const int64_t n_pos = (u_end - u_begin) * NCH;
-    int64_t pf_tile = -1;  // tile whose entry pf_info holds
-    TileInfo pf_info{};
-    auto prefetch = [&](int64_t lin) {
-      if (lane != 0 || lin >= n_pos) return;
-      const int64_t pu = u_begin + lin / NCH, pch = lin % NCH;
-      if (pu / NB != pf_tile) {
-        pf_tile = pu / NB;
-        pf_info = tile_info<NT>(p, pf_tile);
-      }
-      const TileInfo& pt = pf_info;
-      const int64_t prow = static_cast<int64_t>(pt.expert) * p.N + (pu % NB) * unit_rows;
-#pragma unroll
-      for (int m = 0; m < NMAT; ++m) {
-        const int32_t ry = static_cast<int32_t>(prow + (p.pair ? kRows * m : 0));
-        if (p.code3d) {
-          tma_prefetch_l2_3d(&p.tmap[m], 0, ry, static_cast<int32_t>(pch * C::BOXES));
-        } else {
-#pragma unroll
-          for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_prefetch_l2_2d(&p.tmap[m],
-                               static_cast<int32_t>(pch * (C::CHUNK_ROW_BYTES / 4)) + bx * 32, ry);
-        }
-        if (p.sb_tma) {
-          tma_prefetch_l2_2d(&p.tmap_sb[m][0], static_cast<int32_t>(pch * C::KB_PER_CHUNK), ry);
-          tma_prefetch_l2_2d(&p.tmap_sb[m][1], static_cast<int32_t>(pch * C::KB_PER_CHUNK), ry);
-        }
-      }
-    };
-    for (int64_t lin = 0; lin < kPrefetchAhead; ++lin) prefetch(lin);
     uint32_t it = 0;
     bool aborted = false;
     int64_t cur_tile = -1;
@@ -286,7 +248,6 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
                             static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
           }
         }
-        prefetch(static_cast<int64_t>(it) + kPrefetchAhead);
         if (p.sb_tma) continue;
         // scales and biases: [mat][s|b][16 rows][KB_PER_CHUNK] bf16
         const int64_t kb0 = ch * C::KB_PER_CHUNK;

@@ -21,9 +21,14 @@ from inputs import (bf16_bits, decode_tokens, decode_weights, dense_projections,
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["qmv", "tc"])
+@pytest.fixture(params=["qmv", "tc", "auto"])
 def kernel(request, monkeypatch):
-    monkeypatch.setenv("QMOE_FORCE_KERNEL", request.param)
+    """Kernel choice: forced streaming, forced tensor-core, or the library's own plan
+    (chosen from the most rows one expert can receive)."""
+    if request.param == "auto":
+        monkeypatch.delenv("QMOE_FORCE_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("QMOE_FORCE_KERNEL", request.param)
     return request.param
 
 
@@ -211,6 +216,19 @@ def test_switch_glu_prefill(gpu_lib, kernel, T, mode):
         assert np.array_equal(inv, w_inv)
         assert_close(f"prefill sorted T={T}", ys[torch.from_numpy(inv.astype(np.int64)).cuda()],
                      want.reshape(T * d["top_k"], -1))
+
+
+@pytest.mark.parametrize("T", [40, 331])
+def test_switch_glu_prefill_8bit_g128(gpu_lib, kernel, T):
+    """8-bit group-128 prefill SwitchGLU with Zipf-skewed routing: the down projection's
+    rows (K = 512) hold only 4 groups, so on the tensor-core path their scales and
+    biases arrive by 1-D bulk copies of whole 128-row blocks."""
+    q = gpu_lib
+    d = prefill_layer(2, T, group=128, bits=8)
+    W = [qweight(*d[k], 128, 8) for k in ("up", "gate", "down")]
+    want, _ = _switch_oracle(d["x"], d["idx"], d["up"], d["gate"], d["down"], 128, 8)
+    y = q.qmoe_switch_glu(dev_bf16(d["x"]), dev_u32(d["idx"]), *W, mode=0)
+    assert_close(f"prefill 8-bit g128 T={T}", y, want)
 
 
 _PREFILL = {}
