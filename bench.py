@@ -440,6 +440,37 @@ def run_block(q, dev, peaks):
     return out
 
 
+def run_combine(q, dev, peaks):
+    """The one-pass combine (fp32 sum, one rounding) and the stock-tail combine (bf16
+    rounding at each step) on expert-sorted outputs of hidden 2048, top-8, with a gated
+    shared term.  Each must read top_k + 1 rows (and x for the gate dot, or one logit)
+    and write one row per token; reported against the HBM peak."""
+    import torch
+    from gpu_util import dev_bf16, dev_f32, dev_u32
+    from inputs import normal_bf16
+    hbm = peaks["hbm_gbs"] if peaks else 6650.0
+    Hh, K = 2048, TOP_K
+    out = {}
+    for T in (128, 331, 2048, 4096, 16384):
+        rng = np.random.default_rng(T)
+        y = dev_bf16(normal_bf16(rng, (T * K, Hh)))
+        inv = dev_u32(rng.permutation(T * K).astype(np.uint32))
+        sc = dev_f32((rng.random((T, K)) / K).astype(np.float32))
+        sh, x = dev_bf16(normal_bf16(rng, (T, Hh))), dev_bf16(normal_bf16(rng, (T, Hh)))
+        wsg = dev_bf16(normal_bf16(rng, (Hh,), 1 / np.sqrt(Hh)))
+        z = dev_bf16(normal_bf16(rng, (T,)))
+        ob = torch.empty((T, Hh), dtype=torch.bfloat16, device=dev)
+        row = Hh * 2
+        t_one = _graph_time(lambda: q.qmoe_moe_combine(y, inv, sc, sh, x, wsg, out=ob))
+        t_stock = _graph_time(lambda: q.qmoe_moe_combine_stock(y, inv, sc, sh, z, out=ob))
+        b_one = T * ((K + 3) * row + K * 8) + row          # y rows, shared, x, out; inv+scores; w
+        b_stock = T * ((K + 2) * row + K * 8 + 2)           # y rows, shared, out; inv+scores; z
+        out[f"T{T}"] = {
+            "one_pass_us": 1e3 * t_one, "one_pass_frac_hbm": b_one / (t_one * 1e-3) / 1e9 / hbm,
+            "stock_us": 1e3 * t_stock, "stock_frac_hbm": b_stock / (t_stock * 1e-3) / 1e9 / hbm}
+    return out
+
+
 # ---------------------------------------------------------------------- ours
 def main():
     p = argparse.ArgumentParser()
@@ -667,6 +698,7 @@ def main():
         prefill = run_prefill(q, [int(t) for t in args.prefill_tokens.split(",") if t], dev,
                               peaks)
 
+    combine = run_combine(q, dev, peaks) if not args.no_block else None
     dense = run_dense(q, dev, peaks) if not args.no_dense else None
     block = run_block(q, dev, peaks) if not args.no_block else None
 
@@ -692,7 +724,7 @@ def main():
             "config": dict(CONFIG, experts=args.experts), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches,
             "decode_isolated": isolated, "prefill": prefill, "dense_qmm": dense,
-            "moe_block": block,
+            "moe_block": block, "combine": combine,
             "hbm_frac_of_measured": value / hbm_peak,
         }
         print(json.dumps(line), flush=True)

@@ -254,6 +254,31 @@ QMOE_API int qmoe_moe_combine(const qmoe_bf16* y_sorted, const uint32_t* inv_ord
                      int64_t T, int top_k, int64_t H, qmoe_bf16* out, int* d_status,
                      qmoe_stream stream);
 
+/*
+ * qmoe_moe_combine_stock -- the same tail with the stock block's rounding, in one pass
+ * ([P5] Motivation: the stock block unsorts the expert outputs, multiplies by the
+ * scores and sums over top_k, each step writing a bf16 tensor, then adds the gated
+ * shared expert; the combine reproduces that rounding).  Reading of the steps:
+ *   s_k = bf16(scores[t,k])
+ *   p_k = bf16(y_sorted[inv_order[t*top_k+k]] * s_k)     (exact fp32 product)
+ *   r   = bf16(p_0 + ... + p_{top_k-1})                  (fp32 sum in k order)
+ *   g   = bf16(float(sigmoid(z[t])))                     (sigmoid in fp64; 1 if no z)
+ *   out[t] = bf16(r + bf16(g * shared[t]))
+ *   y_sorted [T*top_k, H] bf16; inv_order [T*top_k] uint32; scores [T, top_k] float32
+ *   shared [T, H] bf16 or NULL (no shared term); shared_gate_logit [T] bf16 (each
+ *   token's shared-gate projection z) or NULL for gate 1; out [T, H] bf16.
+ * The result is fixed to the bit by these steps and does not depend on the other
+ * tokens of the call.  inv_order entries >= T*top_k contribute zero and flag
+ * QMOE_DEV_BAD_INDEX.  Errors: QMOE_ERR_ARG (T < 0, top_k <= 0, H <= 0, null or
+ * unaligned tensors, shared_gate_logit without shared), QMOE_ERR_UNSUPPORTED (H not a
+ * multiple of 8), QMOE_ERR_CUDA (launch failure).
+ */
+QMOE_API int qmoe_moe_combine_stock(const qmoe_bf16* y_sorted, const uint32_t* inv_order,
+                                    const float* scores, const qmoe_bf16* shared,
+                                    const qmoe_bf16* shared_gate_logit, int64_t T, int top_k,
+                                    int64_t H, qmoe_bf16* out, int* d_status,
+                                    qmoe_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

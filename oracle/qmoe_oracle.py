@@ -31,7 +31,7 @@ import numpy as np
 __all__ = [
     "bf16_from_f32", "f32_from_bf16", "pack_codes", "unpack_codes", "quantize",
     "dequantize", "qmm", "gather_qmm", "sort_by_expert", "tile_table",
-    "silu", "switch_glu", "moe_combine", "sigmoid",
+    "silu", "switch_glu", "moe_combine", "moe_combine_stock", "sigmoid",
 ]
 
 
@@ -336,3 +336,44 @@ def moe_combine(y_sorted, inv_order, scores, shared=None, x=None, w_shared_gate=
         out += gate[:, None] * sh
     return out
 
+
+def _bf16_round(v: np.ndarray) -> np.ndarray:
+    """float32 values rounded to bf16 (round to nearest even), returned as float32."""
+    return f32_from_bf16(bf16_from_f32(np.asarray(v, np.float32)))
+
+
+def moe_combine_stock(y_sorted, inv_order, scores, shared=None, shared_gate_logit=None):
+    """The MoE block tail step by step, each step rounded to bf16 as the stock block
+    materialises it ([P5] Motivation: unsort to token order, multiply by the scores,
+    sum over top_k, each writing a bf16 tensor, then add the shared expert).
+
+    Reading of the steps (the page names them, not their arithmetic):
+      s_k   = bf16(scores[t, k])                        (routing scores as bf16)
+      p_k   = bf16(y_sorted[inv_order[t*top_k + k]] * s_k)   (fp32 product, exact)
+      r     = bf16(p_0 + p_1 + ... + p_{top_k-1})       (fp32 sum in k order)
+      g     = bf16(float32(sigmoid(z_t)))               (z_t: bf16 gate logit, sigmoid
+                                                          in fp64; g = 1 without logits)
+      out   = bf16(r + bf16(g * shared[t]))             (fp32 product and sum)
+    Every operand of a product is bf16, so each fp32 product is exact and every
+    rounding point is fixed: the result is defined to the bit.  ``y_sorted``,
+    ``shared``, ``shared_gate_logit``: bf16 bit patterns; ``scores`` float32
+    ``[T, top_k]``.  Returns bf16 bits ``[T, H]``.
+    """
+    ys = f32_from_bf16(np.asarray(y_sorted, np.uint16))
+    sc = _bf16_round(np.asarray(scores, np.float32))
+    T, top_k = sc.shape
+    inv = np.asarray(inv_order, np.int64).reshape(T, top_k)
+    r = np.zeros((T, ys.shape[1]), np.float32)
+    for k in range(top_k):
+        p = _bf16_round(ys[inv[:, k]] * sc[:, k:k + 1])
+        r = (r + p).astype(np.float32)
+    r = _bf16_round(r)
+    if shared is None:
+        return bf16_from_f32(r)
+    sh = f32_from_bf16(np.asarray(shared, np.uint16))
+    if shared_gate_logit is None:
+        g = np.ones((T, 1), np.float32)
+    else:
+        z = f32_from_bf16(np.asarray(shared_gate_logit, np.uint16)).astype(np.float64)
+        g = _bf16_round((1.0 / (1.0 + np.exp(-z))).astype(np.float32)).reshape(T, 1)
+    return bf16_from_f32((r + _bf16_round(g * sh)).astype(np.float32))

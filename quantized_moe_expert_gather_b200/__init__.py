@@ -22,7 +22,8 @@ __all__ = [
     "QmoeError", "load", "library_path", "qmoe_status_string", "qmoe_launch_count", "qmoe_timing_enable", "qmoe_timing_read",
     "qmoe_quantize", "qmoe_dequantize", "qmoe_qmm", "qmoe_gather_qmm",
     "qmoe_gather_qmm_workspace_size", "qmoe_gather_qmm_noalloc", "qmoe_sort_by_expert", "qmoe_tile_table",
-    "qmoe_switch_glu", "qmoe_switch_glu_workspace_size", "qmoe_moe_combine", "QWeight",
+    "qmoe_switch_glu", "qmoe_switch_glu_workspace_size", "qmoe_moe_combine",
+    "qmoe_moe_combine_stock", "QWeight",
     "QMOE_DEV_BAD_INDEX", "QMOE_DEV_TIMEOUT", "EXPORTED",
 ]
 
@@ -67,6 +68,7 @@ _SIGS = {
                                ctypes.POINTER(_QWeight), ctypes.POINTER(_QWeight), _i32, _p, _sz,
                                _p, _p, _p, _p]),
     "qmoe_moe_combine": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i32, _i64, _p, _p, _p]),
+    "qmoe_moe_combine_stock": (_i32, [_p, _p, _p, _p, _p, _i64, _i32, _i64, _p, _p, _p]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -342,5 +344,21 @@ def qmoe_moe_combine(y_sorted, inv_order, scores, shared=None, x=None, w_shared_
     out = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=y_sorted.device)
     _check("qmoe_moe_combine", load().qmoe_moe_combine(
         _ptr(y_sorted), _ptr(inv_order), _ptr(scores), _ptr(shared), _ptr(x), _ptr(w_shared_gate),
+        T, top_k, H, _ptr(out), _ptr(status), _stream()))
+    return out
+
+
+def qmoe_moe_combine_stock(y_sorted, inv_order, scores, shared=None, shared_gate_logit=None,
+                           out=None, status=None):
+    """The MoE tail with the stock block's bf16 rounding at every step: out[t] =
+    bf16(bf16(sum_k bf16(y_sorted[inv_order[t*top_k+k]] * bf16(scores[t,k])))
+    + bf16(bf16(sigmoid(z[t])) * shared[t])), z = shared_gate_logit (bf16 [T])."""
+    _need(y_sorted, "y_sorted", _BF16)
+    _need(scores, "scores", (torch.float32,))
+    T, top_k = scores.shape
+    H = y_sorted.shape[-1]
+    out = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=y_sorted.device)
+    _check("qmoe_moe_combine_stock", load().qmoe_moe_combine_stock(
+        _ptr(y_sorted), _ptr(inv_order), _ptr(scores), _ptr(shared), _ptr(shared_gate_logit),
         T, top_k, H, _ptr(out), _ptr(status), _stream()))
     return out

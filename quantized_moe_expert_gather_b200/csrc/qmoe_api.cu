@@ -426,4 +426,19 @@ int qmoe_moe_combine(const qmoe_bf16* y_sorted, const uint32_t* inv_order, const
                                     top_k, H, out, d_status, static_cast<cudaStream_t>(stream)));
 }
 
+int qmoe_moe_combine_stock(const qmoe_bf16* y_sorted, const uint32_t* inv_order,
+                           const float* scores, const qmoe_bf16* shared,
+                           const qmoe_bf16* shared_gate_logit, int64_t T, int top_k, int64_t H,
+                           qmoe_bf16* out, int* d_status, qmoe_stream stream) {
+  if (T < 0 || top_k <= 0 || H <= 0) return QMOE_ERR_ARG;
+  if (H % 8 != 0) return QMOE_ERR_UNSUPPORTED;
+  if (shared_gate_logit != nullptr && shared == nullptr) return QMOE_ERR_ARG;
+  if (T == 0) return QMOE_OK;
+  if (!y_sorted || !inv_order || !scores || !out) return QMOE_ERR_ARG;
+  if (!aligned16(y_sorted) || !aligned16(out) || (shared && !aligned16(shared))) return QMOE_ERR_ARG;
+  return cuda_status(launch_combine_stock(y_sorted, inv_order, scores, shared, shared_gate_logit,
+                                          T, top_k, H, out, d_status,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

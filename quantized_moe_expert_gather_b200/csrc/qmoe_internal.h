@@ -107,5 +107,10 @@ cudaError_t launch_combine(const uint16_t* y_sorted, const uint32_t* inv_order,
                            const float* scores, const uint16_t* shared, const uint16_t* x,
                            const uint16_t* w_sg, int64_t T, int top_k, int64_t H, uint16_t* out,
                            int* d_status, cudaStream_t stream);
+// The same tail with the stock block's bf16 rounding points (see qmoe_moe_combine_stock).
+cudaError_t launch_combine_stock(const uint16_t* y_sorted, const uint32_t* inv_order,
+                                 const float* scores, const uint16_t* shared,
+                                 const uint16_t* gate_logit, int64_t T, int top_k, int64_t H,
+                                 uint16_t* out, int* d_status, cudaStream_t stream);
 
 }  // namespace qmoe

@@ -262,6 +262,63 @@ def test_moe_combine(gpu_lib, T, gated):
     assert_close(f"combine T={T}", out, want)
 
 
+def _stock_case(T, seed):
+    rng = np.random.default_rng(seed)
+    K, H, E = 8, 2048, 256
+    keys = rng.integers(0, E, size=T * K)
+    _, inv, _ = O.sort_by_expert(keys, E)
+    y_sorted = normal_bf16(rng, (T * K, H))
+    p = rng.random((T, K)).astype(np.float32)
+    scores = (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
+    shared = normal_bf16(rng, (T, H))
+    logits = normal_bf16(rng, (T,), 2.0)
+    return y_sorted, inv.astype(np.uint32), scores, shared, logits
+
+
+@pytest.mark.parametrize("T", [128, 331])
+@pytest.mark.parametrize("variant", ["gated", "ungated", "no_shared"])
+def test_moe_combine_stock_bit_exact(gpu_lib, T, variant):
+    """Stock-tail combine: every rounding point is fixed, so the GPU result equals the
+    oracle's bit for bit (MoE block sizes: top-8, hidden 2048)."""
+    q = gpu_lib
+    y_sorted, inv, scores, shared, logits = _stock_case(T, 100 + T)
+    sh = None if variant == "no_shared" else shared
+    z = logits if variant == "gated" else None
+    want = O.moe_combine_stock(y_sorted, inv, scores, sh, z)
+    out = q.qmoe_moe_combine_stock(dev_bf16(y_sorted), dev_u32(inv), dev_f32(scores),
+                                   None if sh is None else dev_bf16(sh),
+                                   None if z is None else dev_bf16(z))
+    got = host_bits16(out)
+    assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} differ"
+
+
+def test_moe_combine_stock_bad_index_and_batch_invariance(gpu_lib):
+    """An out-of-range position contributes nothing and flags the status word (the
+    same bits as a zero score); a token's output does not depend on the other tokens
+    of the call."""
+    q = gpu_lib
+    T, K = 96, 8
+    y_sorted, inv, scores, shared, logits = _stock_case(T, 7)
+    bad = inv.copy()
+    bad[5 * K + 3] = T * K + 11
+    zeroed = scores.copy()
+    zeroed[5, 3] = 0.0
+    want = O.moe_combine_stock(y_sorted, inv, zeroed, shared, logits)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = q.qmoe_moe_combine_stock(dev_bf16(y_sorted), dev_u32(bad), dev_f32(scores),
+                                   dev_bf16(shared), dev_bf16(logits), status=status)
+    assert np.array_equal(host_bits16(out), want)
+    assert int(status.item()) & q.QMOE_DEV_BAD_INDEX
+    full = host_bits16(q.qmoe_moe_combine_stock(dev_bf16(y_sorted), dev_u32(inv), dev_f32(scores),
+                                                dev_bf16(shared), dev_bf16(logits)))
+    a, b = 17, 60  # tokens a..b-1 on their own: their rows, in k order, positions 0..
+    rows = inv.reshape(T, K)[a:b].reshape(-1).astype(np.int64)
+    sub = q.qmoe_moe_combine_stock(dev_bf16(y_sorted[rows]),
+                                   dev_u32(np.arange((b - a) * K, dtype=np.uint32)),
+                                   dev_f32(scores[a:b]), dev_bf16(shared[a:b]), dev_bf16(logits[a:b]))
+    assert np.array_equal(host_bits16(sub), full[a:b])
+
+
 def test_moe_block_prefill_with_shared_expert(gpu_lib):
     """MoE block: routed experts in expert order + shared SwiGLU + sigmoid gate, one
     combine pass (T = 128)."""

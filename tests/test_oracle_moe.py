@@ -107,3 +107,73 @@ def test_combine_shared_gate_closed_forms():
     x0[:, 0] = bf16_bits(np.float32(60.0))
     big = O.moe_combine(y, inv, zeros, shared, x0, w0)
     assert np.allclose(big, O.f32_from_bf16(shared).astype(np.float64), rtol=1e-20, atol=1e-25)
+
+
+# ------------------------------------------------------------- stock-tail combine
+def _bf16_of(values):
+    return bf16_bits(np.asarray(values, np.float32))
+
+
+def test_stock_combine_top1_unit_score_is_the_unsort():
+    """top_k = 1, score 1, no shared term: every rounding is exact, so the result is
+    the expert-sorted rows put back in token order, bit for bit."""
+    rng = np.random.default_rng(11)
+    T, H = 6, 16
+    y = _bf16_of(rng.standard_normal((T, H)))
+    inv = rng.permutation(T).astype(np.uint32)
+    out = O.moe_combine_stock(y, inv, np.ones((T, 1), np.float32))
+    assert np.array_equal(out, y[inv.astype(np.int64)])
+
+
+def test_stock_combine_equals_exact_combine_when_every_step_is_exact():
+    """Small integer rows, power-of-two scores and a shared term gated by sigmoid(0) =
+    1/2: every product and partial sum is a bf16 value, so the stepwise result equals
+    the fp64 combine exactly."""
+    rng = np.random.default_rng(12)
+    T, top_k, H = 5, 4, 16
+    y = _bf16_of(rng.integers(-7, 8, size=(T * top_k, H)))
+    inv = rng.permutation(T * top_k).astype(np.uint32)
+    scores = rng.choice(np.float32([0.25, 0.5, 1.0]), size=(T, top_k)).astype(np.float32)
+    shared = _bf16_of(rng.integers(-6, 7, size=(T, H)))
+    z = _bf16_of(np.zeros(T))
+    got = O.moe_combine_stock(y, inv, scores, shared, z)
+    # gate 1/2 in the fp64 combine: x . w_shared_gate = 0
+    want = O.moe_combine(y, inv, scores, shared, _bf16_of(np.ones((T, H))), _bf16_of(np.zeros(H)))
+    assert np.array_equal(got, _bf16_of(want))
+
+
+def test_stock_combine_within_rounding_bound_of_exact_combine():
+    """Random rows: the stepwise result differs from the fp64 combine by at most the
+    roundings it performs (unit roundoff u = 2^-8 of bf16): scores and products
+    (2u per term), the top_k sum (u) and the final add (u)."""
+    rng = np.random.default_rng(13)
+    T, top_k, H = 16, 8, 64
+    y = _bf16_of(rng.standard_normal((T * top_k, H)))
+    inv = rng.permutation(T * top_k).astype(np.uint32)
+    p = rng.random((T, top_k)).astype(np.float32)
+    scores = (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
+    shared = _bf16_of(rng.standard_normal((T, H)))
+    got = O.f32_from_bf16(O.moe_combine_stock(y, inv, scores, shared)).astype(np.float64)
+    want = O.moe_combine(y, inv, scores, shared)
+    yf = O.f32_from_bf16(y).astype(np.float64)[inv.astype(np.int64)].reshape(T, top_k, H)
+    terms = np.abs(yf * scores.astype(np.float64)[:, :, None]).sum(axis=1)
+    u = 2.0 ** -8
+    bound = 3.1 * u * terms + 1.1 * u * (np.abs(want) + np.abs(O.f32_from_bf16(shared)))
+    err = np.abs(got - want)
+    assert np.all(err <= bound + 1e-30)
+    assert err.max() > 0  # the steps do round
+
+
+def test_stock_combine_gate_closed_forms():
+    """Zero scores leave the gated shared term: logit 0 gives sigmoid 1/2, which halves
+    bf16 values exactly; logit 30 gives a sigmoid that rounds to 1 in float32."""
+    rng = np.random.default_rng(14)
+    T, top_k, H = 4, 2, 16
+    y = _bf16_of(rng.standard_normal((T * top_k, H)))
+    inv = np.arange(T * top_k, dtype=np.uint32)
+    zero = np.zeros((T, top_k), np.float32)
+    shared = _bf16_of(rng.standard_normal((T, H)))
+    half = O.moe_combine_stock(y, inv, zero, shared, _bf16_of(np.zeros(T)))
+    assert np.array_equal(half, _bf16_of(O.f32_from_bf16(shared) / 2))
+    one = O.moe_combine_stock(y, inv, zero, shared, _bf16_of(np.full(T, 30.0)))
+    assert np.array_equal(one, shared)
