@@ -471,6 +471,31 @@ def run_combine(q, dev, peaks):
     return out
 
 
+def run_gather_mm(q, dev, peaks):
+    """Unquantized gather_mm (bf16 weights, the tensor-core kernel without its dequant
+    stage) on the prefill expert projection: hidden 2048 -> 512, 256 experts, Zipf-skewed
+    top-8 routing, x broadcast over each token's experts.  TFLOP/s against the bf16 peak."""
+    import torch
+    from gpu_util import dev_bf16, dev_u32
+    from inputs import normal_bf16, prefill_routing
+    bf16_peak = peaks["bf16_tflops"] if peaks else 1590.0
+    E, K, N = 256, 2048, 512
+    rng = np.random.default_rng(21)
+    w = dev_bf16(normal_bf16(rng, (E, N, K), 1 / np.sqrt(K)))
+    out = {}
+    for T in (4096, 16384):
+        idx, _ = prefill_routing(0, T, E, TOP_K)
+        x = dev_bf16(normal_bf16(rng, (T, 1, K)))
+        rhs = dev_u32(idx.reshape(-1).astype(np.uint32))
+        B = T * TOP_K
+        ws = torch.empty(q.qmoe_gather_mm_workspace_size(B, 1, E, N, K), dtype=torch.uint8, device=dev)
+        y = torch.empty((B, 1, N), dtype=torch.bfloat16, device=dev)
+        t = _graph_time(lambda: q.qmoe_gather_mm(x, w, None, rhs, out=y, workspace=ws))
+        tf = 2.0 * B * N * K / (t * 1e-3) / 1e12
+        out[f"T{T}"] = {"ms": t, "tflops": tf, "frac_bf16_peak": tf / bf16_peak}
+    return out
+
+
 # ---------------------------------------------------------------------- ours
 def main():
     p = argparse.ArgumentParser()
@@ -699,6 +724,7 @@ def main():
                               peaks)
 
     combine = run_combine(q, dev, peaks) if not args.no_block else None
+    gmm = run_gather_mm(q, dev, peaks) if not args.no_block else None
     dense = run_dense(q, dev, peaks) if not args.no_dense else None
     block = run_block(q, dev, peaks) if not args.no_block else None
 
@@ -724,7 +750,7 @@ def main():
             "config": dict(CONFIG, experts=args.experts), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches,
             "decode_isolated": isolated, "prefill": prefill, "dense_qmm": dense,
-            "moe_block": block, "combine": combine,
+            "moe_block": block, "combine": combine, "gather_mm_bf16": gmm,
             "hbm_frac_of_measured": value / hbm_peak,
         }
         print(json.dumps(line), flush=True)

@@ -240,6 +240,28 @@ QMOE_API int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_
                     uint32_t* inv_order, int* d_status, qmoe_stream stream);
 
 /*
+ * qmoe_gather_mm -- the unquantized gathered matmul ([P2] Description and Proposed
+ * changes: gather_mm over rows routed to experts, tiles cut per expert from offsets of
+ * rhs_indices, every tile running one K loop against one expert):
+ *   y[b, m, :] = x[lhs[b], m, :] . W[rhs[b]]^T
+ *   x   [x_batches, M, K] bf16;  w [E, N, K] bf16 (row n of expert e at (e*N + n)*K)
+ *   lhs_indices, rhs_indices, B, sorted_indices as in qmoe_gather_qmm
+ *   y   [B, M, N] bf16.  fp32 accumulation on the tensor cores, one rounding.
+ * Routed rows are sorted by expert into 128-row tiles (the tensor-core kernel
+ * without the dequant stage).  K must be a multiple of 64 (QMOE_ERR_UNSUPPORTED);
+ * x, w and y 16-byte aligned (QMOE_ERR_ARG); workspace at least
+ * qmoe_gather_mm_workspace_size() bytes (QMOE_ERR_WORKSPACE).  Rows with an index
+ * >= E (or a bad lhs) are zeroed and flag QMOE_DEV_BAD_INDEX.
+ */
+QMOE_API size_t qmoe_gather_mm_workspace_size(int64_t B, int64_t M, int64_t E, int64_t N,
+                                              int64_t K);
+QMOE_API int qmoe_gather_mm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
+                            const qmoe_bf16* w, int64_t E, int64_t N,
+                            const uint32_t* lhs_indices, const uint32_t* rhs_indices, int64_t B,
+                            int sorted_indices, void* workspace, size_t workspace_bytes,
+                            qmoe_bf16* y, int* d_status, qmoe_stream stream);
+
+/*
  * qmoe_moe_combine -- one-pass MoE combine ([P5] Summary / Motivation):
  *   out[t] = sum_k scores[t,k] * y_sorted[inv_order[t*top_k+k]]
  *            + sigmoid(x[t] . w_shared_gate) * shared[t]

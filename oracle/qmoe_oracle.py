@@ -30,7 +30,7 @@ import numpy as np
 
 __all__ = [
     "bf16_from_f32", "f32_from_bf16", "pack_codes", "unpack_codes", "quantize",
-    "dequantize", "qmm", "gather_qmm", "sort_by_expert", "tile_table",
+    "dequantize", "qmm", "gather_qmm", "gather_mm", "sort_by_expert", "tile_table",
     "silu", "switch_glu", "moe_combine", "moe_combine_stock", "sigmoid",
 ]
 
@@ -217,6 +217,38 @@ def gather_qmm(x, packed, scales, biases, group: int, bits: int,
         wd = dequantize(packed[e], scales[e], biases[e], group, bits).astype(np.float64)
         for b in np.nonzero(rhs == e)[0]:
             out[b] = xf[lhs[b]] @ wd.T
+    return out
+
+
+def gather_mm(x, w, lhs_indices=None, rhs_indices=None) -> np.ndarray:
+    """Unquantized gathered matmul ([P2] Description: the gather_mm whose row tiles the
+    page reorganises).
+
+    ``x``: bf16 ``[x_batches, M, K]``; ``w``: bf16 ``[E, N, K]``.  Batch b of the result
+    is ``x[lhs[b]] . w[rhs[b]]^T``, with the index defaults of :func:`gather_qmm`.
+    Returns fp64 ``[B, M, N]``.
+    """
+    x = np.asarray(x)
+    w = np.asarray(w)
+    E, xb = w.shape[0], x.shape[0]
+    if lhs_indices is None and rhs_indices is None:
+        B = max(xb, E)
+        lhs = np.arange(B) % xb if xb == B else np.zeros(B, np.int64)
+        rhs = np.arange(B) % E if E == B else np.zeros(B, np.int64)
+    else:
+        rhs = np.asarray(rhs_indices, np.int64).reshape(-1) if rhs_indices is not None else None
+        lhs = np.asarray(lhs_indices, np.int64).reshape(-1) if lhs_indices is not None else None
+        if lhs is None:
+            B = rhs.size
+            lhs = (np.arange(B) * xb) // B
+        if rhs is None:
+            B = lhs.size
+            rhs = (np.arange(B) * E) // B
+        assert lhs.size == rhs.size
+    xf = _as_f32(x).astype(np.float64)
+    out = np.empty((lhs.size, x.shape[1], w.shape[1]), np.float64)
+    for b in range(lhs.size):
+        out[b] = xf[lhs[b]] @ _as_f32(w[rhs[b]]).astype(np.float64).T
     return out
 
 

@@ -23,7 +23,7 @@ __all__ = [
     "qmoe_quantize", "qmoe_dequantize", "qmoe_qmm", "qmoe_gather_qmm",
     "qmoe_gather_qmm_workspace_size", "qmoe_gather_qmm_noalloc", "qmoe_sort_by_expert", "qmoe_tile_table",
     "qmoe_switch_glu", "qmoe_switch_glu_workspace_size", "qmoe_moe_combine",
-    "qmoe_moe_combine_stock", "QWeight",
+    "qmoe_moe_combine_stock", "qmoe_gather_mm", "qmoe_gather_mm_workspace_size", "QWeight",
     "QMOE_DEV_BAD_INDEX", "QMOE_DEV_TIMEOUT", "EXPORTED",
 ]
 
@@ -69,6 +69,9 @@ _SIGS = {
                                _p, _p, _p, _p]),
     "qmoe_moe_combine": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i32, _i64, _p, _p, _p]),
     "qmoe_moe_combine_stock": (_i32, [_p, _p, _p, _p, _p, _i64, _i32, _i64, _p, _p, _p]),
+    "qmoe_gather_mm_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i64]),
+    "qmoe_gather_mm": (_i32, [_p, _i64, _i64, _i64, _p, _i64, _i64, _p, _p, _i64, _i32, _p, _sz,
+                              _p, _p, _p]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -362,3 +365,36 @@ def qmoe_moe_combine_stock(y_sorted, inv_order, scores, shared=None, shared_gate
         _ptr(y_sorted), _ptr(inv_order), _ptr(scores), _ptr(shared), _ptr(shared_gate_logit),
         T, top_k, H, _ptr(out), _ptr(status), _stream()))
     return out
+
+
+def qmoe_gather_mm_workspace_size(B: int, M: int, E: int, N: int, K: int) -> int:
+    return int(load().qmoe_gather_mm_workspace_size(B, M, E, N, K))
+
+
+def qmoe_gather_mm(x, w, lhs_indices=None, rhs_indices=None, sorted_indices: bool = False,
+                   out=None, workspace=None, status=None):
+    """Unquantized gather_mm: y[b] = x[lhs[b]] . W[rhs[b]]^T for x [x_batches, M, K] bf16
+    and W [E, N, K] bf16; 1-D index tensors.  Returns [B, M, N] bf16."""
+    _need(x, "x", _BF16)
+    _need(w, "w", _BF16)
+    xb, M, K = x.shape
+    E, N = w.shape[0], w.shape[1]
+    if lhs_indices is not None:
+        _need(lhs_indices, "lhs_indices", _IDX)
+    if rhs_indices is not None:
+        _need(rhs_indices, "rhs_indices", _IDX)
+    if lhs_indices is None and rhs_indices is None:
+        B = max(xb, E)
+    elif rhs_indices is not None:
+        B = rhs_indices.numel()
+    else:
+        B = lhs_indices.numel()
+    if lhs_indices is not None and lhs_indices.numel() != B:
+        raise ValueError("lhs_indices and rhs_indices have different sizes")
+    y = out if out is not None else torch.empty((B, M, N), dtype=torch.bfloat16, device=x.device)
+    need = qmoe_gather_mm_workspace_size(B, M, E, N, K)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check("qmoe_gather_mm", load().qmoe_gather_mm(
+        _ptr(x), xb, M, K, _ptr(w), E, N, _ptr(lhs_indices), _ptr(rhs_indices), B,
+        int(bool(sorted_indices)), _ptr(ws), ws.numel(), _ptr(y), _ptr(status), _stream()))
+    return y

@@ -268,6 +268,70 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   return cuda_status(launch_qmv(a, s));
 }
 
+size_t qmoe_gather_mm_workspace_size(int64_t B, int64_t M, int64_t E, int64_t N, int64_t K) {
+  return qmoe_gather_qmm_workspace_size(B, M, E, N, K);
+}
+
+int qmoe_gather_mm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K, const qmoe_bf16* w,
+                   int64_t E, int64_t N, const uint32_t* lhs_indices, const uint32_t* rhs_indices,
+                   int64_t B, int sorted_indices, void* workspace, size_t workspace_bytes,
+                   qmoe_bf16* y, int* d_status, qmoe_stream stream) {
+  (void)sorted_indices;  // a promise about rhs; the expert sort makes it unnecessary
+  if (K <= 0 || x_batches <= 0 || M < 0 || B < 0 || E <= 0 || N <= 0) return QMOE_ERR_ARG;
+  if (K % 64 != 0) return QMOE_ERR_UNSUPPORTED;
+  if (B == 0 || M == 0) return QMOE_OK;
+  if (!x || !w || !y) return QMOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return QMOE_ERR_ARG;
+  if (workspace == nullptr || workspace_bytes < qmoe_gather_mm_workspace_size(B, M, E, N, K))
+    return QMOE_ERR_WORKSPACE;
+  const int64_t R = B * M;
+  Carver cv(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255)));
+  RouteBufs rb = carve_route(cv, R, E, true);
+  uint16_t* x_sorted = cv.take<uint16_t>(R * K);
+
+  GemmArgs a;
+  a.w[0] = QWeight{reinterpret_cast<const uint32_t*>(w), nullptr, nullptr};
+  a.nmat = 1;
+  a.E = E;
+  a.N = N;
+  a.K = K;
+  a.group = 64;  // no groups: bf16 weights
+  a.bits = 16;
+  a.y = y;
+  a.x = x_sorted;
+  a.x_rows = R;
+  a.dst_row = rb.order;
+  a.tiles = rb.tiles;
+  a.num_tiles = rb.num_tiles;
+  a.bm = kTcBm;
+  a.max_tiles = max_tiles_for(R, E, kTcBm);
+  a.d_status = d_status;
+
+  RouteArgs ra;
+  ra.rhs = rhs_indices;
+  ra.lhs = lhs_indices;
+  ra.B = B;
+  ra.M = M;
+  ra.x_batches = x_batches;
+  ra.E = E;
+  ra.bm = kTcBm;
+  ra.order = rb.order;
+  ra.inv_order = rb.inv;
+  ra.offsets = rb.offsets;
+  ra.src_row = rb.src_row;
+  ra.tiles = rb.tiles;
+  ra.num_tiles = rb.num_tiles;
+  ra.max_tiles = a.max_tiles;
+  ra.zero_out = y;
+  ra.zero_cols = N;
+  ra.zero_by_pos = false;
+  ra.d_status = d_status;
+  auto s = static_cast<cudaStream_t>(stream);
+  if (launch_route(ra, rb.route_ws, s) != cudaSuccess) return QMOE_ERR_CUDA;
+  if (launch_gather_rows(x, rb.src_row, R, K, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
+  return cuda_status(launch_qmm_tc(a, s));
+}
+
 size_t qmoe_sort_by_expert_workspace_size(int64_t R, int64_t E) {
   return route_workspace_bytes(std::max<int64_t>(R, 0), std::max<int64_t>(E, 1)) + 256;
 }

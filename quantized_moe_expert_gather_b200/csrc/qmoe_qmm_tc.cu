@@ -50,15 +50,18 @@ struct TcCfg {
 #define QMOE_TC_S1_4BIT 5
 #define QMOE_TC_S2_4BIT 2
 #endif
-  static constexpr int S1 = BITS == 4 ? QMOE_TC_S1_4BIT : 4;     // activation + packed-code ring
-  static constexpr int S2 = BITS == 4 ? QMOE_TC_S2_4BIT : 2;     // dequantised-weight ring
+  // BITS == 16: unquantized bf16 weights, copied by TMA straight into the weight ring
+  // (no packed codes, scales or dequant warps); that ring takes their space.
+  static constexpr bool WBF16 = BITS == 16;
+  static constexpr int S1 = BITS == 4 ? QMOE_TC_S1_4BIT : (WBF16 ? 5 : 4);  // activation ring
+  static constexpr int S2 = BITS == 4 ? QMOE_TC_S2_4BIT : (WBF16 ? 4 : 2);  // weight ring
   static constexpr int A_BYTES = kBM * kBK * 2;                  // 16 KB
   static constexpr int P_ROW = kBK * BITS / 8;                   // packed bytes per row per stage
-  static constexpr int PK = 128 / P_ROW;                         // stages per packed-code load
-  static constexpr int SP = 2;                                   // packed-code ring
+  static constexpr int PK = WBF16 ? 1 : 128 / P_ROW;             // stages per packed-code load
+  static constexpr int SP = WBF16 ? 0 : 2;                       // packed-code ring
   static constexpr int P_SLOT = 2 * kBM * 128;                   // two stacks, 128 B per row
   static constexpr int B_BYTES = 2 * kBN * kBK * 2;              // two stacks, bf16
-  static constexpr int SB_BYTES = 2 * 2 * kBM * kSbGroups * 2;   // [stack][s|b][row][8]
+  static constexpr int SB_BYTES = WBF16 ? 0 : 2 * 2 * kBM * kSbGroups * 2;  // [stack][s|b][row][8]
   static constexpr int OFF_A = 0;
   static constexpr int OFF_P = OFF_A + S1 * A_BYTES;
   static constexpr int OFF_B = OFF_P + SP * P_SLOT;
@@ -71,7 +74,8 @@ struct TcCfg {
 
 struct alignas(64) TcParams {
   CUtensorMap tm_a;        // activation rows [x_rows, K] bf16, box {64, 128}, 128B swizzle
-  CUtensorMap tm_w[2];     // packed codes [E*N, K*bits/32] u32, box {32, 128}, 128B swizzle
+  CUtensorMap tm_w[2];     // packed codes [E*N, K*bits/32] u32, box {32, 128}, 128B swizzle;
+                           // bf16 weights [E*N, K], box {64, 128}, 128B swizzle
   CUtensorMap tm_sb[2][2]; // scales / biases [E*N, K/group] bf16, box {8, 128}
   uint16_t* y;
   const uint32_t* dst_row;
@@ -240,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
       mbar_init(&emptyP[s], kDqWarps);
     }
     for (int s = 0; s < kS2; ++s) {
-      mbar_init(&full2[s], kDqWarps);
+      mbar_init(&full2[s], C::WBF16 ? 1 : kDqWarps);  // TMA tx, or the dequant warps
       mbar_init(&empty2[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -294,45 +298,57 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         const int64_t wrow = static_cast<int64_t>(tl.expert) * p.N + n0;
         for (int64_t ks = 0; ks < KS; ++ks) {
           if (*abort_flag) { ab = true; break; }
-          if (sb_first(ks)) {
-            const uint32_t e = sbit & 1;
-            if (!mbar_wait(&empty_sb[e], ((sbit >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
-            if constexpr (SB_WHOLE) {
-              // rows wrow.. of one stack are contiguous: [128 rows][sb_groups] per array
-              const uint32_t bytes = kBM * p.sb_groups * 2;
-              mbar_arrive_expect_tx(&full_sb[e], 4 * bytes);
-#pragma unroll
-              for (int m = 0; m < 2; ++m) {
-                const int64_t r0 = wrow + (p.pair ? kBN * m : 0);
-#pragma unroll
-                for (int arr = 0; arr < 2; ++arr)
-                  bulk_load(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
-                            (arr ? p.biases[m] : p.scales[m]) + r0 * p.sb_groups, bytes, &full_sb[e]);
-              }
-            } else {
-              mbar_arrive_expect_tx(&full_sb[e], C::SB_BYTES);
-              const int32_t gx = static_cast<int32_t>(ks * kBK / GS);
-#pragma unroll
-              for (int m = 0; m < 2; ++m)
-#pragma unroll
-                for (int arr = 0; arr < 2; ++arr)
-                  tma_load_2d(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
-                              &p.tm_sb[m][arr], &full_sb[e], gx,
-                              static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
-            }
-            ++sbit;
-          }
-          if (ks % C::PK == 0) {
-            // packed codes of the next PK stages: 128 bytes of each row, 128B-swizzled
-            const uint32_t ps = pbit % C::SP;
-            if (!mbar_wait(&emptyP[ps], ((pbit / C::SP) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
-            mbar_arrive_expect_tx(&fullP[ps], C::P_SLOT);
+          if constexpr (C::WBF16) {
+            // bf16 weight tiles, 128 rows x 64 k per stack, straight into the weight ring
+            const uint32_t s2 = it % kS2;
+            if (!mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+            mbar_arrive_expect_tx(&full2[s2], C::B_BYTES);
 #pragma unroll
             for (int m = 0; m < 2; ++m)
-              tma_load_2d(smem + C::OFF_P + ps * C::P_SLOT + m * kBM * 128, &p.tm_w[m], &fullP[ps],
-                          static_cast<int32_t>(ks * kBK * BITS / 32),
+              tma_load_2d(smem + C::OFF_B + s2 * C::B_BYTES + m * kBN * kBK * 2, &p.tm_w[m],
+                          &full2[s2], static_cast<int32_t>(ks * kBK),
                           static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
-            ++pbit;
+          } else {
+            if (sb_first(ks)) {
+              const uint32_t e = sbit & 1;
+              if (!mbar_wait(&empty_sb[e], ((sbit >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+              if constexpr (SB_WHOLE) {
+                // rows wrow.. of one stack are contiguous: [128 rows][sb_groups] per array
+                const uint32_t bytes = kBM * p.sb_groups * 2;
+                mbar_arrive_expect_tx(&full_sb[e], 4 * bytes);
+  #pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                  const int64_t r0 = wrow + (p.pair ? kBN * m : 0);
+  #pragma unroll
+                  for (int arr = 0; arr < 2; ++arr)
+                    bulk_load(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
+                              (arr ? p.biases[m] : p.scales[m]) + r0 * p.sb_groups, bytes, &full_sb[e]);
+                }
+              } else {
+                mbar_arrive_expect_tx(&full_sb[e], C::SB_BYTES);
+                const int32_t gx = static_cast<int32_t>(ks * kBK / GS);
+  #pragma unroll
+                for (int m = 0; m < 2; ++m)
+  #pragma unroll
+                  for (int arr = 0; arr < 2; ++arr)
+                    tma_load_2d(smem + C::OFF_SB + e * C::SB_BYTES + (m * 2 + arr) * kBM * kSbGroups * 2,
+                                &p.tm_sb[m][arr], &full_sb[e], gx,
+                                static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
+              }
+              ++sbit;
+            }
+            if (ks % C::PK == 0) {
+              // packed codes of the next PK stages: 128 bytes of each row, 128B-swizzled
+              const uint32_t ps = pbit % C::SP;
+              if (!mbar_wait(&emptyP[ps], ((pbit / C::SP) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+              mbar_arrive_expect_tx(&fullP[ps], C::P_SLOT);
+  #pragma unroll
+              for (int m = 0; m < 2; ++m)
+                tma_load_2d(smem + C::OFF_P + ps * C::P_SLOT + m * kBM * 128, &p.tm_w[m], &fullP[ps],
+                            static_cast<int32_t>(ks * kBK * BITS / 32),
+                            static_cast<int32_t>(wrow + (p.pair ? kBN * m : 0)));
+              ++pbit;
+            }
           }
           const uint32_t s1 = it % kS1;
           if (!mbar_wait(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
@@ -348,9 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
         for (uint32_t k = first; k < it; ++k) mbar_wait(&full1[k % kS1], (k / kS1) & 1, nullptr);
         const uint32_t sfirst = sbit > 2u ? sbit - 2 : 0u;
         for (uint32_t k = sfirst; k < sbit; ++k) mbar_wait(&full_sb[k & 1], (k >> 1) & 1, nullptr);
-        const uint32_t pfirst = pbit > static_cast<uint32_t>(C::SP) ? pbit - C::SP : 0u;
-        for (uint32_t k = pfirst; k < pbit; ++k)
-          mbar_wait(&fullP[k % C::SP], (k / C::SP) & 1, nullptr);
+        if constexpr (C::WBF16) {
+          const uint32_t bfirst = it > static_cast<uint32_t>(kS2) ? it - kS2 : 0u;
+          for (uint32_t k = bfirst; k < it; ++k) mbar_wait(&full2[k % kS2], (k / kS2) & 1, nullptr);
+        } else {
+          const uint32_t pfirst = pbit > static_cast<uint32_t>(C::SP) ? pbit - C::SP : 0u;
+          for (uint32_t k = pfirst; k < pbit; ++k)
+            mbar_wait(&fullP[k % C::SP], (k / C::SP) & 1, nullptr);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -398,76 +419,78 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
       }
     }
   } else if (warp >= kDqWarp0) {
-    // ------------------------------------------------------------------- dequant
-    // Thread dq handles half-rows hr = dq and dq + 256 of the 512 (stack, row, half)
-    // half-rows of a stage: consecutive lanes read consecutive 16-byte pieces of the
-    // packed tile and write distinct swizzled 16-byte chunks (no bank conflicts).
-    const int dq = threadIdx.x - kDqWarp0 * 32;  // 0..255
-    constexpr int HALF = C::P_ROW / 2;           // packed bytes per half-row: 16 or 32
-    uint32_t it = 0, sbit = 0, pbit = 0;
-    for (int64_t u = u_begin; u < u_end; u += u_step) {
-      for (int64_t ks = 0; ks < KS; ++ks, ++it) {
-        if (*abort_flag) break;
-        const uint32_t e = sbit & 1;
-        if (sb_first(ks) &&
-            !mbar_wait(&full_sb[e], (sbit >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
-        const uint32_t ps = pbit % C::SP, s2 = it % kS2;
-        if (ks % C::PK == 0 &&
-            !mbar_wait(&fullP[ps], (pbit / C::SP) & 1, p.d_status)) { *abort_flag = 1; break; }
-        if (!mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
-        const int pj = static_cast<int>(ks % C::PK);  // stage inside the packed rows
-        const int gin = sb_whole ? static_cast<int>(ks * kBK / GS)
-                                 : static_cast<int>((ks * kBK / GS) % kSbGroups);
+    if constexpr (!C::WBF16) {  // bf16 weights arrive by TMA: nothing to dequantise
+      // ------------------------------------------------------------------- dequant
+      // Thread dq handles half-rows hr = dq and dq + 256 of the 512 (stack, row, half)
+      // half-rows of a stage: consecutive lanes read consecutive 16-byte pieces of the
+      // packed tile and write distinct swizzled 16-byte chunks (no bank conflicts).
+      const int dq = threadIdx.x - kDqWarp0 * 32;  // 0..255
+      constexpr int HALF = C::P_ROW / 2;           // packed bytes per half-row: 16 or 32
+      uint32_t it = 0, sbit = 0, pbit = 0;
+      for (int64_t u = u_begin; u < u_end; u += u_step) {
+        for (int64_t ks = 0; ks < KS; ++ks, ++it) {
+          if (*abort_flag) break;
+          const uint32_t e = sbit & 1;
+          if (sb_first(ks) &&
+              !mbar_wait(&full_sb[e], (sbit >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
+          const uint32_t ps = pbit % C::SP, s2 = it % kS2;
+          if (ks % C::PK == 0 &&
+              !mbar_wait(&fullP[ps], (pbit / C::SP) & 1, p.d_status)) { *abort_flag = 1; break; }
+          if (!mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+          const int pj = static_cast<int>(ks % C::PK);  // stage inside the packed rows
+          const int gin = sb_whole ? static_cast<int>(ks * kBK / GS)
+                                   : static_cast<int>((ks * kBK / GS) % kSbGroups);
 #pragma unroll
-        for (int rep = 0; rep < 2; ++rep) {
-          const int hr = dq + 256 * rep;          // (stack, row, half)
-          const int m = hr / (2 * kBM), row = (hr / 2) % kBM, half = hr & 1;
-          const uint16_t* sbp = reinterpret_cast<const uint16_t*>(smem + C::OFF_SB + e * C::SB_BYTES) +
-                                (m * 2) * kBM * kSbGroups + row * sb_stride;
-          const uint16_t* bbp = sbp + kBM * kSbGroups;
-          // packed row: 128 bytes, 16-byte chunk c stored at chunk c ^ (row & 7)
-          const uint8_t* prow = smem + C::OFF_P + ps * C::P_SLOT + (m * kBM + row) * 128;
-          const int pc = (pj * C::P_ROW + half * HALF) / 16;  // first chunk of this half-row
-          uint8_t* brow = smem + C::OFF_B + s2 * C::B_BYTES + (m * kBN + row) * (kBK * 2);
-          // codes 32*half .. 32*half+31 of this row's 64
-          const int gj = gin + (GS == 32 ? half : 0);
-          if constexpr (BITS == 4) {
-            const uint4 pw = *reinterpret_cast<const uint4*>(prow + ((pc ^ (row & 7)) << 4));
-            const uint32_t w[4] = {pw.x, pw.y, pw.z, pw.w};
-            const uint16_t sv = sbp[gj], bv = bbp[gj];
-            const __nv_bfloat162 s2v = __halves2bfloat162(__ushort_as_bfloat16(sv), __ushort_as_bfloat16(sv));
-            const __nv_bfloat162 b2v = __halves2bfloat162(__ushort_as_bfloat16(bv), __ushort_as_bfloat16(bv));
+          for (int rep = 0; rep < 2; ++rep) {
+            const int hr = dq + 256 * rep;          // (stack, row, half)
+            const int m = hr / (2 * kBM), row = (hr / 2) % kBM, half = hr & 1;
+            const uint16_t* sbp = reinterpret_cast<const uint16_t*>(smem + C::OFF_SB + e * C::SB_BYTES) +
+                                  (m * 2) * kBM * kSbGroups + row * sb_stride;
+            const uint16_t* bbp = sbp + kBM * kSbGroups;
+            // packed row: 128 bytes, 16-byte chunk c stored at chunk c ^ (row & 7)
+            const uint8_t* prow = smem + C::OFF_P + ps * C::P_SLOT + (m * kBM + row) * 128;
+            const int pc = (pj * C::P_ROW + half * HALF) / 16;  // first chunk of this half-row
+            uint8_t* brow = smem + C::OFF_B + s2 * C::B_BYTES + (m * kBN + row) * (kBK * 2);
+            // codes 32*half .. 32*half+31 of this row's 64
+            const int gj = gin + (GS == 32 ? half : 0);
+            if constexpr (BITS == 4) {
+              const uint4 pw = *reinterpret_cast<const uint4*>(prow + ((pc ^ (row & 7)) << 4));
+              const uint32_t w[4] = {pw.x, pw.y, pw.z, pw.w};
+              const uint16_t sv = sbp[gj], bv = bbp[gj];
+              const __nv_bfloat162 s2v = __halves2bfloat162(__ushort_as_bfloat16(sv), __ushort_as_bfloat16(sv));
+              const __nv_bfloat162 b2v = __halves2bfloat162(__ushort_as_bfloat16(bv), __ushort_as_bfloat16(bv));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int c = 4 * half + j;             // 16-byte chunk = codes 8c .. 8c+7
-              *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = dequant_word4(w[j], s2v, b2v);
-            }
-          } else {
-            const uint4 pa = *reinterpret_cast<const uint4*>(prow + ((pc ^ (row & 7)) << 4));
-            const uint4 pb = *reinterpret_cast<const uint4*>(prow + (((pc + 1) ^ (row & 7)) << 4));
-            const uint32_t w[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-            const float sv = bf16_to_f32(sbp[gj]), bv = bf16_to_f32(bbp[gj]);
+              for (int j = 0; j < 4; ++j) {
+                const int c = 4 * half + j;             // 16-byte chunk = codes 8c .. 8c+7
+                *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = dequant_word4(w[j], s2v, b2v);
+              }
+            } else {
+              const uint4 pa = *reinterpret_cast<const uint4*>(prow + ((pc ^ (row & 7)) << 4));
+              const uint4 pb = *reinterpret_cast<const uint4*>(prow + (((pc + 1) ^ (row & 7)) << 4));
+              const uint32_t w[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+              const float sv = bf16_to_f32(sbp[gj]), bv = bf16_to_f32(bbp[gj]);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int c = 4 * half + j;             // two 8-bit words per chunk
-              const uint2 a = dequant_word8(w[2 * j], sv, bv);
-              const uint2 b = dequant_word8(w[2 * j + 1], sv, bv);
-              *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+              for (int j = 0; j < 4; ++j) {
+                const int c = 4 * half + j;             // two 8-bit words per chunk
+                const uint2 a = dequant_word8(w[2 * j], sv, bv);
+                const uint2 b = dequant_word8(w[2 * j + 1], sv, bv);
+                *reinterpret_cast<uint4*>(brow + ((c ^ (row & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+              }
             }
           }
+          fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
+          __syncwarp();
+          const bool p_done = ks % C::PK == C::PK - 1 || ks == KS - 1;
+          if (lane == 0) {
+            mbar_arrive(&full2[s2]);
+            if (p_done) mbar_arrive(&emptyP[ps]);
+            if (sb_last(ks)) mbar_arrive(&empty_sb[e]);
+          }
+          if (p_done) ++pbit;
+          if (sb_last(ks)) ++sbit;
         }
-        fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
-        __syncwarp();
-        const bool p_done = ks % C::PK == C::PK - 1 || ks == KS - 1;
-        if (lane == 0) {
-          mbar_arrive(&full2[s2]);
-          if (p_done) mbar_arrive(&emptyP[ps]);
-          if (sb_last(ks)) mbar_arrive(&empty_sb[e]);
-        }
-        if (p_done) ++pbit;
-        if (sb_last(ks)) ++sbit;
+        if (*abort_flag) break;
       }
-      if (*abort_flag) break;
     }
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------------------------ epilogue
@@ -569,6 +592,7 @@ cudaError_t launch_tc(const TcParams& prm, cudaStream_t stream) {
 }  // namespace
 
 bool qmm_tc_supported(const GemmArgs& a) {
+  if (a.bits == 16) return a.K % kBK == 0 && a.x_rows > 0;  // unquantized bf16 weights
   if (a.bits != 4 && a.bits != 8) return false;
   if (a.K % kBK != 0) return false;
   const int64_t gpr = a.K / a.group;
@@ -587,6 +611,24 @@ cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream) {
   cudaError_t e = make_tmap_2d_bf16(&prm.tm_a, a.x, a.K, a.x_rows, kBK, kBM, /*swizzle128=*/true);
   if (e != cudaSuccess) return e;
   prm.pair = a.nmat == 2 ? 0 : 1;
+  if (a.bits == 16) {
+    // bf16 weights [E*N, K]: 128 rows x 64 k per box, 128B-swizzled like the
+    // dequantised tiles
+    for (int m = 0; m < 2; ++m) {
+      const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
+      e = make_tmap_2d_bf16(&prm.tm_w[m], wm.codes, a.K, a.E * a.N, kBK, kBM, /*swizzle128=*/true);
+      if (e != cudaSuccess) return e;
+    }
+    prm.y = a.y;
+    prm.dst_row = a.dst_row;
+    prm.tiles = a.tiles;
+    prm.num_tiles = a.num_tiles;
+    prm.dense_rows = a.dense_rows;
+    prm.N = a.N;
+    prm.K = a.K;
+    prm.d_status = a.d_status;
+    return launch_tc_sb<16, 64, false>(prm, stream);
+  }
   const int64_t words = a.K * a.bits / 32;
   const int64_t gpr = a.K / a.group;
   for (int m = 0; m < 2; ++m) {

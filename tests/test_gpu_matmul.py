@@ -16,7 +16,8 @@ import oracle as O
 from gpu_util import (assert_close, dev_bf16, dev_f32, dev_u32, host_bits16, host_u32,
                       qweight, select_experts)
 from inputs import (bf16_bits, decode_tokens, decode_weights, dense_projections,
-                    dense_weight_f32, normal_bf16, prefill_layer, random_qweight, tiny_gather)
+                    dense_weight_f32, normal_bf16, prefill_layer, prefill_routing, random_qweight,
+                    tiny_gather)
 
 pytestmark = pytest.mark.gpu
 
@@ -238,6 +239,68 @@ def _prefill(T):
     if T not in _PREFILL:
         _PREFILL[T] = prefill_layer(0, T)
     return _PREFILL[T]
+
+
+# ------------------------------------------------------------------- gather_mm
+GATHER_MM_CASES = [  # (x_batches, M, K, E, N, B)
+    (300, 1, 512, 8, 200, 300),   # rows across three 128-row tiles; N not a multiple of 128
+    (40, 1, 256, 5, 384, 320),    # x broadcast over 8 experts per token
+    (3, 7, 128, 4, 64, 3),        # several rows per batch, one tile
+]
+
+
+@pytest.mark.parametrize("xb,M,K,E,N,B", GATHER_MM_CASES)
+def test_gather_mm(gpu_lib, xb, M, K, E, N, B):
+    """Unquantized gather_mm on the tensor-core kernel (no dequant stage) against the
+    oracle; sorted and unsorted indices give the same bits."""
+    q = gpu_lib
+    rng = np.random.default_rng(1000 + K + N)
+    w = normal_bf16(rng, (E, N, K), 1 / np.sqrt(K))
+    x = normal_bf16(rng, (xb, M, K))
+    rhs = rng.integers(0, E, size=B).astype(np.uint32)
+    lhs = None if xb != B else rng.permutation(B).astype(np.uint32)
+    want = O.gather_mm(x, w, lhs, rhs)
+    got = q.qmoe_gather_mm(dev_bf16(x), dev_bf16(w), None if lhs is None else dev_u32(lhs),
+                           dev_u32(rhs))
+    assert_close(f"gather_mm {xb}x{M}x{K} E={E} N={N} B={B}", got, want)
+    if lhs is None:
+        lhs_b = ((np.arange(B) * xb) // B).astype(np.uint32)
+        order = np.argsort(rhs, kind="stable")
+        srt = q.qmoe_gather_mm(dev_bf16(x), dev_bf16(w), dev_u32(lhs_b[order]),
+                               dev_u32(rhs[order]), sorted_indices=True)
+        assert np.array_equal(host_bits16(srt), host_bits16(got)[order])
+
+
+def test_gather_mm_bad_index_zeroes_row(gpu_lib):
+    q = gpu_lib
+    rng = np.random.default_rng(5)
+    E, N, K, B = 4, 128, 256, 150
+    w = normal_bf16(rng, (E, N, K), 1 / np.sqrt(K))
+    x = normal_bf16(rng, (B, 1, K))
+    rhs = rng.integers(0, E, size=B).astype(np.uint32)
+    rhs[17] = E + 3
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = q.qmoe_gather_mm(dev_bf16(x), dev_bf16(w), None, dev_u32(rhs), status=status)
+    assert int(status.item()) & q.QMOE_DEV_BAD_INDEX
+    assert not torch.any(got[17].float() != 0)
+    keep = np.arange(B) != 17
+    want = O.gather_mm(x[keep], w, None, rhs[keep])
+    assert_close("gather_mm rows with valid indices", got[torch.from_numpy(keep).cuda()], want)
+
+
+def test_gather_mm_prefill_shape(gpu_lib):
+    """Prefill-shaped unquantized expert projection: hidden 2048 -> 512, 256 experts,
+    Zipf-skewed top-8 routing of 512 tokens (x broadcast over each token's experts)."""
+    q = gpu_lib
+    T, E, K, N = 512, 256, 2048, 512
+    rng = np.random.default_rng(9)
+    idx, _ = prefill_routing(3, T, E, 8)
+    w = normal_bf16(rng, (E, N, K), 1 / np.sqrt(K))
+    x = normal_bf16(rng, (T, 1, K))
+    rhs = idx.reshape(-1).astype(np.uint32)
+    got = q.qmoe_gather_mm(dev_bf16(x), dev_bf16(w), None, dev_u32(rhs))
+    want = O.gather_mm(x, w, None, rhs)
+    assert_close("gather_mm prefill shape", got, want)
 
 
 # --------------------------------------------------------------------- combine

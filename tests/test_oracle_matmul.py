@@ -95,3 +95,38 @@ def test_gather_qmm_sorted_and_unsorted_indices_agree_bitwise():
     unsorted = O.gather_qmm(x, w, s, b, group, bits, lhs, rhs)
     sorted_ = O.gather_qmm(x, w, s, b, group, bits, lhs[perm], rhs[perm])
     assert np.array_equal(sorted_, unsorted[perm])
+
+
+# ------------------------------------------------------------------ gather_mm
+def test_gather_mm_matches_exact_rational_brute_force():
+    """Unquantized gather_mm against exact rational dot products of the bf16 values."""
+    rng = np.random.default_rng(0x91)
+    E, N, K, M = 3, 5, 48, 2
+    w = bf16_bits(rng.standard_normal((E, N, K)).astype(np.float32))
+    x = bf16_bits(rng.standard_normal((4, M, K)).astype(np.float32))
+    wf, xf = O.f32_from_bf16(w), O.f32_from_bf16(x)
+    lhs, rhs = [3, 0, 2, 0], [1, 2, 0, 1]
+    got = O.gather_mm(x, w, lhs, rhs)
+    assert got.shape == (4, M, N)
+    for j, (l, r) in enumerate(zip(lhs, rhs)):
+        for m in range(M):
+            for n in range(N):
+                val, mag = _exact_dot(xf[l, m], [Fraction(float(v)) for v in wf[r, n]])
+                assert abs(got[j, m, n] - float(val)) <= 1e-12 * float(mag) + 1e-300
+
+
+def test_gather_mm_equals_gather_qmm_on_exactly_dequantised_weights():
+    """With scale 1/4 and bias -2 every dequantised weight q/4 - 2 is a bf16 value, so
+    gather_mm over those bf16 weights and gather_qmm over the codes agree exactly
+    (index defaults and broadcast of x over the weights included)."""
+    rng = np.random.default_rng(0x92)
+    E, N, K, M, group, bits = 4, 6, 64, 3, 32, 4
+    codes = rng.integers(0, 16, size=(E, N, K))
+    packed = O.pack_codes(codes.reshape(E * N, K), bits).reshape(E, N, -1)
+    s = bf16_bits(np.full((E, N, K // group), 0.25, np.float32))
+    b = bf16_bits(np.full((E, N, K // group), -2.0, np.float32))
+    w = bf16_bits((codes * 0.25 - 2.0).astype(np.float32))
+    x = bf16_bits(rng.standard_normal((2, M, K)).astype(np.float32))
+    rhs = [3, 1, 1, 0, 2]
+    assert np.array_equal(O.gather_mm(x, w, None, rhs), O.gather_qmm(x, packed, s, b, group, bits, None, rhs))
+    assert np.array_equal(O.gather_mm(x[:1], w), O.gather_qmm(x[:1], packed, s, b, group, bits))
