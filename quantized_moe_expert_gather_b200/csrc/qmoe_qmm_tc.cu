@@ -18,7 +18,7 @@
 //         each of the 128 rows per stack (128B-swizzled, own two-slot ring); every 8
 //         groups, the scales and biases;
 //   5     MMA issuer: owns 512 TMEM columns (two double-buffered unit accumulators),
-//         one thread issues tcgen05.mma kind::f16 (M=128, N=128, K=16) and commits to
+//         one thread issues tcgen05.mma kind::f16 (M=128, N=256, K=16) and commits to
 //         mbarriers;
 //   6-13  dequant: one thread per (stack, row) turns 64 packed codes into bf16
 //         q*scale + bias (one rounding) and writes them in the 128B-swizzled K-major
@@ -172,9 +172,12 @@ __device__ __forceinline__ uint64_t sw128_desc(const void* smem_tile) {
          (uint64_t(1) << 46) /* descriptor version */ | (uint64_t(2) << 61) /* 128B swizzle */;
 }
 
-// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, M=128, N=128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
-                            (uint32_t(kBM >> 4) << 24);
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, M=128,
+// N=256: one MMA covers both weight tiles of a stage (they are contiguous in shared
+// memory with the same 1024-byte 8-row stride) and both accumulators (adjacent TMEM
+// columns).
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            (uint32_t((2 * kBN) >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
 
 __device__ __forceinline__ uint32_t bf16x2_of(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
@@ -400,11 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t adesc = sw128_desc(a_t) + 2 * kk;  // +32 bytes along k
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-              const uint64_t bdesc = sw128_desc(b_t + m * kBN * kBK * 2) + 2 * kk;
-              tc_mma(d0 + m * kBN, adesc, bdesc, kIdesc, (ks | kk) != 0 ? 1u : 0u);
-            }
+            const uint64_t bdesc = sw128_desc(b_t) + 2 * kk;  // both stacks' 128-row tiles
+            tc_mma(d0, adesc, bdesc, kIdesc, (ks | kk) != 0 ? 1u : 0u);
           }
           issued = true;
           tc_commit(&empty1[s1]);
