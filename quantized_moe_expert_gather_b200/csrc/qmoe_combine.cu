@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
   __shared__ float score_sh[kKChunk];
   const int64_t t = blockIdx.x;
   const int tid = threadIdx.x;
+  griddep_wait();  // the expert outputs come from the kernel before this one
+  griddep_launch_dependents();
   if (tid == 0) prof_start(prof);
   const int64_t nvec = H / 8;
   const int64_t v = static_cast<int64_t>(blockIdx.y) * kThreads + tid;  // this thread's vector
@@ -142,6 +144,8 @@ __global__ void __launch_bounds__(kThreads) combine_stock_kernel(
   __shared__ float gate_sh;
   const int64_t t = blockIdx.x;
   const int tid = threadIdx.x;
+  griddep_wait();  // the expert outputs come from the kernel before this one
+  griddep_launch_dependents();
   if (tid == 0) {
     prof_start(prof);
     float g = 1.0f;
@@ -224,9 +228,9 @@ cudaError_t launch_combine_stock(const uint16_t* y_sorted, const uint32_t* inv_o
   if (slices > 65535) return cudaErrorInvalidValue;
   LaunchTimer timer("combine", stream);
   const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>(slices));
-  combine_stock_kernel<<<grid, kThreads, 0, stream>>>(y_sorted, inv_order, scores, shared,
-                                                      gate_logit, T, top_k, H, out, d_status,
-                                                      timer.slot());
+  if (launch_pdl(combine_stock_kernel, grid, dim3(kThreads), 0, stream, y_sorted, inv_order, scores,
+                 shared, gate_logit, T, top_k, H, out, d_status, timer.slot()) != cudaSuccess)
+    return cudaGetLastError();
   count_launch();
   return cudaGetLastError();
 }
@@ -241,8 +245,9 @@ cudaError_t launch_combine(const uint16_t* y_sorted, const uint32_t* inv_order,
   if (slices > 65535) return cudaErrorInvalidValue;
   LaunchTimer timer("combine", stream);
   const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>(slices));
-  combine_kernel<<<grid, kThreads, 0, stream>>>(y_sorted, inv_order, scores, shared, x, w_sg, T,
-                                                top_k, H, out, d_status, timer.slot());
+  if (launch_pdl(combine_kernel, grid, dim3(kThreads), 0, stream, y_sorted, inv_order, scores, shared,
+                 x, w_sg, T, top_k, H, out, d_status, timer.slot()) != cudaSuccess)
+    return cudaGetLastError();
   count_launch();
   return cudaGetLastError();
 }

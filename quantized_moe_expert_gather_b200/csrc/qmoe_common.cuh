@@ -51,6 +51,17 @@ __device__ __forceinline__ void prof_end(Slot* p) {
   if (p != nullptr) atomicMax(&p->end, global_ns());
 }
 
+// --------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the kernel
+// before it on the stream is still running.  griddep_wait() blocks until that kernel has
+// completed and its memory is visible; every read of inputs another kernel produced
+// comes after it (it is a no-op for ordinary launches).  griddep_launch_dependents()
+// lets the next kernel start its own prologue once every CTA of this grid has issued it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- mbarriers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -1,5 +1,6 @@
 // Host-side plumbing: launch counter, SM count cache, TMA descriptor encoding.
 #include <atomic>
+#include <cstdlib>
 #include <cstring>
 #include <cudaTypedefs.h>
 #include <map>
@@ -62,6 +63,14 @@ cudaError_t make_tmap_colblocks(CUtensorMap* map, const void* base, int64_t word
 }  // namespace
 
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("QMOE_PDL");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return on;
+}
 
 namespace {
 struct TimingState {

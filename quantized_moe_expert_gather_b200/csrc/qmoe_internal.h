@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <utility>
 
 #include "../../include/qmoe.h"
 
@@ -12,6 +13,27 @@ namespace qmoe {
 
 void count_launch(int n = 1);
 int sm_count();
+// Programmatic dependent launch on (default) or off (environment QMOE_PDL=0).
+bool pdl_enabled();
+
+// Launches `kernel` with programmatic stream serialization (when enabled): the kernel
+// may run its prologue, up to griddep_wait(), while the previous kernel on the stream
+// finishes.  Inside CUDA graph capture this becomes a programmatic dependency edge.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Device-side timing record of one launch: ~(earliest CTA start) and the latest
 // CTA end, in global-timer nanoseconds, both combined with atomicMax.

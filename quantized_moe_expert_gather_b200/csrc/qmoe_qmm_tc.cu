@@ -259,7 +259,6 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    prof_start(p.prof);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_base_sh, kTmemCols);
@@ -269,6 +268,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_sh;
+  // inputs (tile table, activations) may come from the kernel before this one
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) prof_start(p.prof);
 
   const int64_t KS = p.K / kBK;  // k stages per unit
   // Scale/bias window: one box of 8 groups (KS_SB_BOX stages), or the whole row when it
@@ -578,7 +581,8 @@ cudaError_t launch_tc_sb(TcParams prm, cudaStream_t stream) {
   if (attr_err != cudaSuccess) return attr_err;
   LaunchTimer timer(prm.pair ? "tc" : "tc_glu", stream);
   prm.prof = timer.slot();
-  kern<<<sm_count(), kThreads, C::SMEM + 1024, stream>>>(prm);
+  cudaError_t le = launch_pdl(kern, dim3(sm_count()), dim3(kThreads), C::SMEM + 1024, stream, prm);
+  if (le != cudaSuccess) return le;
   count_launch();
   return cudaGetLastError();
 }

@@ -174,9 +174,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
     }
     *abort_flag = 0;
     fence_mbar_init();
-    prof_start(p.prof);
   }
   __syncthreads();
+  // inputs (tile table, activations) may come from the kernel before this one
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) prof_start(p.prof);
 
   const int64_t KB_TOTAL = p.K / GS;
   const int64_t NCH = (KB_TOTAL + C::KB_PER_CHUNK - 1) / C::KB_PER_CHUNK;
@@ -657,7 +660,9 @@ cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
   if (attr_err != cudaSuccess) return attr_err;
   LaunchTimer timer(prm.pair ? "qmv" : "qmv_glu", stream);
   prm.prof = timer.slot();
-  kern<<<sm_count(), C::THREADS, C::SMEM_BYTES + 1024, stream>>>(prm);
+  cudaError_t le = launch_pdl(kern, dim3(sm_count()), dim3(C::THREADS), C::SMEM_BYTES + 1024,
+                              stream, prm);
+  if (le != cudaSuccess) return le;
   count_launch();
   return cudaGetLastError();
 }

@@ -189,6 +189,8 @@ __device__ void phase_scatter(const RouteDev& d, int64_t chunk) {
 
 __global__ void __launch_bounds__(kChunk) route_count_kernel(RouteDev d) {
   extern __shared__ uint8_t cnt[];
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) prof_start(d.prof);
   phase_count(d, blockIdx.x, cnt);
   __syncthreads();
@@ -196,12 +198,16 @@ __global__ void __launch_bounds__(kChunk) route_count_kernel(RouteDev d) {
 }
 __global__ void __launch_bounds__(kChunk) route_scan_kernel(RouteDev d, int64_t nchunks) {
   __shared__ uint32_t sh[32];
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) prof_start(d.prof);
   phase_scan(d, nchunks, sh);
   __syncthreads();
   if (threadIdx.x == 0) prof_end(d.prof);
 }
 __global__ void __launch_bounds__(kChunk) route_scatter_kernel(RouteDev d) {
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) prof_start(d.prof);
   phase_scatter(d, blockIdx.x);
   __syncthreads();
@@ -218,6 +224,8 @@ __global__ void __launch_bounds__(kChunk) route_fused_kernel(RouteDev d) {
   const int64_t nb = d.E + 1;
   uint8_t* cnt = dyn;
   uint32_t* base = reinterpret_cast<uint32_t*>(dyn + ((32 * nb + 15) & ~int64_t(15)));
+  griddep_wait();  // the indices may come from the kernel before this one
+  griddep_launch_dependents();
   if (tid == 0) prof_start(d.prof);
   for (int64_t i = tid; i < 32 * nb; i += blockDim.x) cnt[i] = 0;
   const int64_t r = tid;
@@ -278,6 +286,8 @@ __global__ void __launch_bounds__(kChunk)
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x,
                                    const uint32_t* __restrict__ src_row, int64_t rows,
                                    int64_t cols, uint16_t* __restrict__ out, ProfSlot* prof) {
+  griddep_wait();  // src_row comes from the route kernel
+  griddep_launch_dependents();
   if (threadIdx.x == 0) prof_start(prof);
   // cols is a multiple of 8: 16-byte vectors.
   const int64_t vec_per_row = cols / 8;
@@ -341,23 +351,29 @@ cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream) {
                            static_cast<int>(fused_bytes));
     LaunchTimer timer("route", stream);
     d.prof = timer.slot();
-    route_fused_kernel<<<1, kChunk, fused_bytes, stream>>>(d);
+    if (launch_pdl(route_fused_kernel, dim3(1), dim3(kChunk), fused_bytes, stream, d) != cudaSuccess)
+      return cudaGetLastError();
     count_launch();
   } else {
     {
       LaunchTimer timer("route", stream);
       d.prof = timer.slot();
-      route_count_kernel<<<static_cast<unsigned>(nchunks), kChunk, cnt_bytes, stream>>>(d);
+      if (launch_pdl(route_count_kernel, dim3(static_cast<unsigned>(nchunks)), dim3(kChunk),
+                     cnt_bytes, stream, d) != cudaSuccess)
+        return cudaGetLastError();
     }
     {
       LaunchTimer timer("route", stream);
       d.prof = timer.slot();
-      route_scan_kernel<<<1, kChunk, 0, stream>>>(d, nchunks);
+      if (launch_pdl(route_scan_kernel, dim3(1), dim3(kChunk), 0, stream, d, nchunks) != cudaSuccess)
+        return cudaGetLastError();
     }
     {
       LaunchTimer timer("route", stream);
       d.prof = timer.slot();
-      route_scatter_kernel<<<static_cast<unsigned>(nchunks), kChunk, 0, stream>>>(d);
+      if (launch_pdl(route_scatter_kernel, dim3(static_cast<unsigned>(nchunks)), dim3(kChunk), 0,
+                     stream, d) != cudaSuccess)
+        return cudaGetLastError();
     }
     count_launch(3);
   }
@@ -380,8 +396,9 @@ cudaError_t launch_gather_rows(const uint16_t* x, const uint32_t* src_row, int64
   const int threads = 256;
   const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 16);
   LaunchTimer timer("gather_rows", stream);
-  gather_rows_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, src_row, rows,
-                                                                            cols, out, timer.slot());
+  if (launch_pdl(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream,
+                 x, src_row, rows, cols, out, timer.slot()) != cudaSuccess)
+    return cudaGetLastError();
   count_launch();
   return cudaGetLastError();
 }
