@@ -67,11 +67,18 @@ constexpr int kTcBm = 128;
 struct Plan {
   bool tc;
   int bm;
+  bool qdec = false;  // streaming on the tensor cores (tiles of 16 rows, rows gathered first)
 };
-Plan plan_for(int64_t R, int64_t E, int64_t max_rows, bool tc_ok) {
+// The streaming kernel on the tensor cores (QMOE_DECODE=qdec) instead of mma.sync.
+bool qdec_requested() {
+  const char* v = std::getenv("QMOE_DECODE");
+  return v != nullptr && std::strcmp(v, "qdec") == 0;
+}
+Plan plan_for(int64_t R, int64_t E, int64_t max_rows, bool tc_ok, bool qdec_ok = false) {
   const Kernel k = forced_kernel();
   const int64_t touched = std::max<int64_t>(1, std::min(E, R));
-  const Plan stream{false, R / touched > 8 ? 16 : 8};
+  Plan stream{false, R / touched > 8 ? 16 : 8};
+  if (qdec_ok && qdec_requested()) stream = Plan{false, 16, true};
   if (!tc_ok || k == Kernel::Qmv) return stream;
   if (k == Kernel::Tc || max_rows > 16) return {true, kTcBm};
   return stream;
@@ -181,9 +188,11 @@ int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, const qmoe_bf
   // one weight matrix: tensor cores from 32 rows, else the streaming kernel
   const Kernel k = forced_kernel();
   const bool tc = qmm_tc_supported(a) && (k == Kernel::Tc || (k == Kernel::Auto && M >= 32));
-  a.bm = tc ? kTcBm : (M > 8 ? 16 : 8);
+  const bool qdec = !tc && qdec_requested() && qdec_supported(a);
+  a.bm = tc ? kTcBm : (qdec || M > 8 ? 16 : 8);
   a.max_tiles = (M + a.bm - 1) / a.bm;
   auto s = static_cast<cudaStream_t>(stream);
+  if (qdec) return cuda_status(launch_qdec(a, s));
   return cuda_status(tc ? launch_qmm_tc(a, s) : launch_qmv(a, s));
 }
 
@@ -232,7 +241,10 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   a.d_status = d_status;
   // Any expert may receive every routed row; below one 128-row tile the streaming
   // kernel serves every expert.
-  const Plan pl = plan_for(R, E, R > kTcBm ? R : 16, qmm_tc_supported(a));
+  GemmArgs a_sorted = a;  // as the tensor-core streaming kernel would read x
+  a_sorted.x = x_sorted;
+  a_sorted.src_row = nullptr;
+  const Plan pl = plan_for(R, E, R > kTcBm ? R : 16, qmm_tc_supported(a), qdec_supported(a_sorted));
   a.bm = pl.bm;
   a.max_tiles = max_tiles_for(R, E, pl.bm);
 
@@ -262,6 +274,12 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
     a.x = x_sorted;  // 128-row tiles over the expert-ordered rows
     a.src_row = nullptr;
     return cuda_status(launch_qmm_tc(a, s));
+  }
+  if (pl.qdec) {
+    if (launch_gather_rows(x, rb.src_row, R, K, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
+    a.x = x_sorted;
+    a.src_row = nullptr;
+    return cuda_status(launch_qdec(a, s));
   }
   a.x = x;  // the streaming kernel reads x through src_row
   a.src_row = rb.src_row;
@@ -436,7 +454,10 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   dn.d_status = d_status;
   // With distinct experts per token one expert receives at most T rows.  The bound only
   // picks the plan: any routing is served correctly by either kernel.
-  const Plan pl = plan_for(R, E, T, qmm_tc_supported(ug) && qmm_tc_supported(dn));
+  GemmArgs ug_sorted = ug;  // as the tensor-core streaming kernel would read x
+  ug_sorted.src_row = nullptr;
+  const Plan pl = plan_for(R, E, T, qmm_tc_supported(ug) && qmm_tc_supported(dn),
+                           qdec_supported(ug_sorted) && qdec_supported(dn));
   ug.bm = dn.bm = pl.bm;
   ug.max_tiles = dn.max_tiles = max_tiles_for(R, E, pl.bm);
 
@@ -466,6 +487,13 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
     ug.src_row = nullptr;
     if (launch_qmm_tc(ug, s) != cudaSuccess) return QMOE_ERR_CUDA;
     return cuda_status(launch_qmm_tc(dn, s));
+  }
+  if (pl.qdec) {
+    if (launch_gather_rows(x, rb.src_row, R, H, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
+    ug.x = x_sorted;
+    ug.src_row = nullptr;
+    if (launch_qdec(ug, s) != cudaSuccess) return QMOE_ERR_CUDA;
+    return cuda_status(launch_qdec(dn, s));
   }
   ug.x = x;
   ug.src_row = rb.src_row;

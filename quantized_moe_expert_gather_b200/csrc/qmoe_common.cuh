@@ -179,6 +179,18 @@ __device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Named barrier that also returns, to every participant, whether any of them passed
+// `pred` true: a decision all of them take together.
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
 
 // --------------------------------------------------------------- warp-level MMA
 // D = A(16x16, row) * B(16x8, col) + C, bf16 inputs, fp32 accumulation.

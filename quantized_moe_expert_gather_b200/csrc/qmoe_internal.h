@@ -121,6 +121,10 @@ struct GemmArgs {
   int* d_status = nullptr;
 };
 cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream);   // tiles of <= 16 rows
+// Tensor-core streaming kernel for few rows per expert (tiles of <= 16 rows): 4-bit codes,
+// activations already in tile order (x_rows rows, src_row null).
+bool qdec_supported(const GemmArgs& a);
+cudaError_t launch_qdec(const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream); // tiles of 128 rows
 bool qmm_tc_supported(const GemmArgs& a);
 

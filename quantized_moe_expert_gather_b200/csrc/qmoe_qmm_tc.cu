@@ -31,6 +31,7 @@
 
 #include "qmoe_common.cuh"
 #include "qmoe_internal.h"
+#include "qmoe_tcgen05.cuh"
 #include "qmoe_tma.h"
 
 namespace qmoe {
@@ -110,68 +111,6 @@ __device__ __forceinline__ Tile tc_tile(const TcParams& p, int64_t j) {
   return t;
 }
 
-// ------------------------------------------------------------- tcgen05 helpers
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulation.
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor of a K-major, 128B-swizzled bf16 tile whose rows are
-// 128 bytes (64 k) and whose 8-row groups are 1024 bytes apart.
-__device__ __forceinline__ uint64_t sw128_desc(const void* smem_tile) {
-  const uint64_t start = (smem_u32(smem_tile) >> 4) & 0x3FFFu;
-  return start | (uint64_t(1) << 16) /* leading offset (unused when swizzled) */ |
-         (uint64_t(1024 >> 4) << 32) /* stride between 8-row groups */ |
-         (uint64_t(1) << 46) /* descriptor version */ | (uint64_t(2) << 61) /* 128B swizzle */;
-}
-
 // Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, M=128,
 // N=256: one MMA covers both weight tiles of a stage (they are contiguous in shared
 // memory with the same 1024-byte 8-row stride) and both accumulators (adjacent TMEM
@@ -180,23 +119,6 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
                             (uint32_t((2 * kBN) >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
 
 __device__ __forceinline__ uint32_t bf16x2_of(float lo, float hi) { return pack_bf16x2(lo, hi); }
-
-// 8 packed 4-bit codes (one word, k ascending) -> 8 bf16 of q*s + b (one rounding each).
-__device__ __forceinline__ uint4 dequant_word4(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
-  const uint32_t ws = w >> 4;
-  const __nv_bfloat162 off = __floats2bfloat162_rn(128.f, 128.f);
-  uint32_t out[4];
-#pragma unroll
-  for (int pp = 0; pp < 4; ++pp) {
-    // byte pp of w (low nibble: code 2pp) -> bits 0..3; byte pp of w>>4 (code 2pp+1) -> 16..19
-    const uint32_t sel = pp | (pp << 4) | ((4 + pp) << 8) | ((4 + pp) << 12);
-    const uint32_t y = and_or(prmt(w, ws, sel), 0x000F000Fu, 0x43004300u);  // 128 + q
-    __nv_bfloat162 q2 = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&y), off);  // exact
-    __nv_bfloat162 v = __hfma2(q2, s2, b2);
-    out[pp] = *reinterpret_cast<uint32_t*>(&v);
-  }
-  return make_uint4(out[0], out[1], out[2], out[3]);
-}
 
 // 4 packed 8-bit codes -> 4 bf16 of q*s + b (fp32 fma, then one rounding to bf16).
 __device__ __forceinline__ uint2 dequant_word8(uint32_t w, float s, float b) {

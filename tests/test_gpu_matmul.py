@@ -22,12 +22,17 @@ from inputs import (bf16_bits, decode_tokens, decode_weights, dense_projections,
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["qmv", "tc", "auto"])
+@pytest.fixture(params=["qmv", "qdec", "tc", "auto"])
 def kernel(request, monkeypatch):
-    """Kernel choice: forced streaming, forced tensor-core, or the library's own plan
-    (chosen from the most rows one expert can receive)."""
+    """Kernel choice: forced streaming (mma.sync, or tcgen05 where it supports the shape),
+    forced tensor-core tiles, or the library's own plan (chosen from the most rows one
+    expert can receive)."""
+    monkeypatch.delenv("QMOE_DECODE", raising=False)
     if request.param == "auto":
         monkeypatch.delenv("QMOE_FORCE_KERNEL", raising=False)
+    elif request.param == "qdec":
+        monkeypatch.setenv("QMOE_FORCE_KERNEL", "qmv")
+        monkeypatch.setenv("QMOE_DECODE", "qdec")
     else:
         monkeypatch.setenv("QMOE_FORCE_KERNEL", request.param)
     return request.param
@@ -179,7 +184,7 @@ def _switch_oracle(x, idx, up, gate, down, group, bits):
 
 
 @pytest.mark.parametrize("M", [1, 4])
-def test_switch_glu_decode_layer(gpu_lib, M):
+def test_switch_glu_decode_layer(gpu_lib, kernel, M):
     """Decode layer at full size: hidden 4096, intermediate 2048, E=288, top-8."""
     q = gpu_lib
     up, gate, down = _decode_weights()
