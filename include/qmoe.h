@@ -137,6 +137,12 @@ QMOE_API int qmoe_dequantize(const uint32_t* codes, const void* scales, const vo
  *   x [M, K] bf16; codes [N, K*bits/32]; scales, biases [N, K/group] bf16;
  *   y [M, N] bf16 (out), fp32 accumulation, one rounding at the end.
  * M = 0 is a no-op.  No workspace.
+ * Ordering: the kernel may begin streaming codes, scales and biases while the kernel
+ * launched just before it on the stream is still running (only x is read after that
+ * kernel has completed).  The weights therefore must not be written by that kernel if
+ * it is one of this library's hot-path kernels (qmm, gather_qmm, switch_glu, combine,
+ * routing); weights written by qmoe_quantize, qmoe_dequantize, a copy or any kernel
+ * outside this library are complete before the weights are read.
  */
 QMOE_API int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, const qmoe_bf16* scales,
              const qmoe_bf16* biases, int64_t N, int64_t K, int group, int bits, qmoe_bf16* y,

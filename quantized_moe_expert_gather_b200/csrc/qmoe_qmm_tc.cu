@@ -18,8 +18,8 @@
 //         each of the 128 rows per stack (128B-swizzled, own two-slot ring); every 8
 //         groups, the scales and biases;
 //   5     MMA issuer: owns 512 TMEM columns (two double-buffered unit accumulators),
-//         one thread issues tcgen05.mma kind::f16 (M=128, N=256, K=16) and commits to
-//         mbarriers;
+//         one elected lane issues tcgen05.mma kind::f16 (M=128, N=256, K=16) and
+//         commits to mbarriers;
 //   6-13  dequant: one thread per (stack, row) turns 64 packed codes into bf16
 //         q*scale + bias (one rounding) and writes them in the 128B-swizzled K-major
 //         layout the MMA descriptors read.
@@ -304,45 +304,55 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      uint32_t it = 0, tc = 0;
-      bool issued = false;
-      for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
-        if (*abort_flag) break;
-        const uint32_t buf = tc & 1;
-        if (!mbar_wait(&tempty[buf], ((tc >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+    // The whole warp walks the loop, so that addresses and descriptors stay
+    // warp-uniform; lane 0 waits and one elected lane (the same one throughout)
+    // issues the MMAs and the commits that track them.
+    uint32_t it = 0, tc = 0;
+    bool issued = false;
+    int ok = 1;
+    for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
+      const uint32_t buf = tc & 1;
+      if (lane == 0) ok = !*abort_flag && mbar_wait(&tempty[buf], ((tc >> 1) & 1) ^ 1, p.d_status);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d0 = tmem_base + buf * (2 * kBN);
+      for (int64_t ks = 0; ks < KS; ++ks, ++it) {
+        const uint32_t s1 = it % kS1, s2 = it % kS2;
+        if (lane == 0)
+          ok = mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) &&
+               mbar_wait(&full2[s2], (it / kS2) & 1, p.d_status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) *abort_flag = 1;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d0 = tmem_base + buf * (2 * kBN);
-        bool ok = true;
-        for (int64_t ks = 0; ks < KS; ++ks, ++it) {
-          const uint32_t s1 = it % kS1, s2 = it % kS2;
-          if (!mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) ||
-              !mbar_wait(&full2[s2], (it / kS2) & 1, p.d_status)) {
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint8_t* a_t = smem + C::OFF_A + s1 * C::A_BYTES;
-          const uint8_t* b_t = smem + C::OFF_B + s2 * C::B_BYTES;
+        const uint64_t a0 = sw128_desc(smem + C::OFF_A + s1 * C::A_BYTES);
+        const uint64_t b0 = sw128_desc(smem + C::OFF_B + s2 * C::B_BYTES);  // both stacks' tiles
+        if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t adesc = sw128_desc(a_t) + 2 * kk;  // +32 bytes along k
-            const uint64_t bdesc = sw128_desc(b_t) + 2 * kk;  // both stacks' 128-row tiles
-            tc_mma(d0, adesc, bdesc, kIdesc, (ks | kk) != 0 ? 1u : 0u);
-          }
-          issued = true;
+          for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes along k per step
+            tc_mma(d0, a0 + 2 * kk, b0 + 2 * kk, kIdesc, (ks | kk) != 0 ? 1u : 0u);
           tc_commit(&empty1[s1]);
           tc_commit(&empty2[s2]);
         }
-        if (!ok) break;
-        tc_commit(&tfull[buf]);
+        __syncwarp();
+        issued = true;
       }
-      if (*abort_flag && issued) {
-        tc_commit(drain);  // completes when every MMA issued so far has finished
-        mbar_wait(drain, 0, nullptr);
-      }
+      if (!ok) break;
+      if (elect_one()) tc_commit(&tfull[buf]);
+      __syncwarp();
     }
+    __syncwarp();
+    const bool leader = elect_one();
+    if (leader && issued && *abort_flag) {
+      tc_commit(drain);  // completes when every MMA issued so far has finished
+      mbar_wait(drain, 0, nullptr);
+    }
+    __syncwarp();
   } else if (warp >= kDqWarp0) {
     if constexpr (!C::WBF16) {  // bf16 weights arrive by TMA: nothing to dequantise
       // ------------------------------------------------------------------- dequant

@@ -176,8 +176,11 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  // inputs (tile table, activations) may come from the kernel before this one
-  griddep_wait();
+  // Inputs (tile table, activations) may come from the kernel before this one.  A dense
+  // launch has no tile table, and its weights are never written by the kernel launched
+  // just before it: there the producer streams weights at once, overlapping the tail of
+  // that kernel, and only the roles that read activations or write y wait.
+  if (!(p.dense_rows > 0 && warp == kConsumerWarps)) griddep_wait();
   griddep_launch_dependents();
   if (threadIdx.x == 0) prof_start(p.prof);
 
