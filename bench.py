@@ -302,13 +302,14 @@ def run_prefill(q, token_counts, dev, peaks, reps=5):
         pf()
         torch.cuda.synchronize()
         split = {k: q.qmoe_timing_read(k)[0] for k in
-                 ("route", "gather_rows", "tc_glu", "tc", "qmv_glu", "qmv", "combine")}
+                 ("route", "gather_rows", "ts_glu", "ts", "tc_glu", "tc", "qmv_glu", "qmv",
+                  "combine")}
         q.qmoe_timing_enable(None)
         flop = T * TOP_K * PREFILL_FLOP_PER_ROW
         tf = flop / (t * 1e-3) / 1e12
         bf16_peak = peaks["bf16_tflops"] if peaks else 1590.0
-        glu_ms = split["tc_glu"] or split["qmv_glu"]
-        dn_ms = split["tc"] or split["qmv"]
+        glu_ms = split["ts_glu"] or split["tc_glu"] or split["qmv_glu"]
+        dn_ms = split["ts"] or split["tc"] or split["qmv"]
         glu_tf = T * TOP_K * 4 * 2048 * 512 / (glu_ms * 1e-3) / 1e12 if glu_ms else None
         dn_tf = T * TOP_K * 2 * 2048 * 512 / (dn_ms * 1e-3) / 1e12 if dn_ms else None
         # bytes the layer must move at least: touched experts' weights, the activations

@@ -68,19 +68,30 @@ struct Plan {
   bool tc;
   int bm;
   bool qdec = false;  // streaming on the tensor cores (tiles of 16 rows, rows gathered first)
+  bool ts = false;    // tensor cores with the weights in tensor memory (tiles of 192 rows)
 };
+// QMOE_PREFILL=tc keeps the tensor-core plan on the kernel that stages dequantised
+// weights in shared memory (tiles of 128 rows) where the tensor-memory one applies.
+bool ts_allowed() {
+  const char* v = std::getenv("QMOE_PREFILL");
+  return v == nullptr || std::strcmp(v, "tc") != 0;
+}
 // The streaming kernel on the tensor cores (QMOE_DECODE=qdec) instead of mma.sync.
 bool qdec_requested() {
   const char* v = std::getenv("QMOE_DECODE");
   return v != nullptr && std::strcmp(v, "qdec") == 0;
 }
-Plan plan_for(int64_t R, int64_t E, int64_t max_rows, bool tc_ok, bool qdec_ok = false) {
+Plan plan_for(int64_t R, int64_t E, int64_t max_rows, bool tc_ok, bool qdec_ok = false,
+              bool ts_ok = false) {
   const Kernel k = forced_kernel();
   const int64_t touched = std::max<int64_t>(1, std::min(E, R));
   Plan stream{false, R / touched > 8 ? 16 : 8};
   if (qdec_ok && qdec_requested()) stream = Plan{false, 16, true};
-  if (!tc_ok || k == Kernel::Qmv) return stream;
-  if (k == Kernel::Tc || max_rows > 16) return {true, kTcBm};
+  if (!(tc_ok || ts_ok) || k == Kernel::Qmv) return stream;
+  if (k == Kernel::Tc || max_rows > 16) {
+    if (ts_ok && ts_allowed()) return Plan{true, kTsTileRows, false, true};
+    if (tc_ok) return Plan{true, kTcBm};
+  }
   return stream;
 }
 
@@ -187,11 +198,14 @@ int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, const qmoe_bf
   a.d_status = d_status;
   // one weight matrix: tensor cores from 32 rows, else the streaming kernel
   const Kernel k = forced_kernel();
-  const bool tc = qmm_tc_supported(a) && (k == Kernel::Tc || (k == Kernel::Auto && M >= 32));
-  const bool qdec = !tc && qdec_requested() && qdec_supported(a);
-  a.bm = tc ? kTcBm : (qdec || M > 8 ? 16 : 8);
+  const bool big = k == Kernel::Tc || (k == Kernel::Auto && M >= 32);
+  const bool ts = big && ts_allowed() && qmm_ts_supported(a);
+  const bool tc = !ts && big && qmm_tc_supported(a);
+  const bool qdec = !ts && !tc && qdec_requested() && qdec_supported(a);
+  a.bm = ts ? kTsTileRows : tc ? kTcBm : (qdec || M > 8 ? 16 : 8);
   a.max_tiles = (M + a.bm - 1) / a.bm;
   auto s = static_cast<cudaStream_t>(stream);
+  if (ts) return cuda_status(launch_qmm_ts(a, s));
   if (qdec) return cuda_status(launch_qdec(a, s));
   return cuda_status(tc ? launch_qmm_tc(a, s) : launch_qmv(a, s));
 }
@@ -244,7 +258,8 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   GemmArgs a_sorted = a;  // as the tensor-core streaming kernel would read x
   a_sorted.x = x_sorted;
   a_sorted.src_row = nullptr;
-  const Plan pl = plan_for(R, E, R > kTcBm ? R : 16, qmm_tc_supported(a), qdec_supported(a_sorted));
+  const Plan pl = plan_for(R, E, R > kTcBm ? R : 16, qmm_tc_supported(a), qdec_supported(a_sorted),
+                           qmm_ts_supported(a_sorted));
   a.bm = pl.bm;
   a.max_tiles = max_tiles_for(R, E, pl.bm);
 
@@ -271,9 +286,9 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   if (launch_route(ra, rb.route_ws, s) != cudaSuccess) return QMOE_ERR_CUDA;
   if (pl.tc) {
     if (launch_gather_rows(x, rb.src_row, R, K, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
-    a.x = x_sorted;  // 128-row tiles over the expert-ordered rows
+    a.x = x_sorted;  // row tiles over the expert-ordered rows
     a.src_row = nullptr;
-    return cuda_status(launch_qmm_tc(a, s));
+    return cuda_status(pl.ts ? launch_qmm_ts(a, s) : launch_qmm_tc(a, s));
   }
   if (pl.qdec) {
     if (launch_gather_rows(x, rb.src_row, R, K, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
@@ -457,7 +472,8 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   GemmArgs ug_sorted = ug;  // as the tensor-core streaming kernel would read x
   ug_sorted.src_row = nullptr;
   const Plan pl = plan_for(R, E, T, qmm_tc_supported(ug) && qmm_tc_supported(dn),
-                           qdec_supported(ug_sorted) && qdec_supported(dn));
+                           qdec_supported(ug_sorted) && qdec_supported(dn),
+                           qmm_ts_supported(ug_sorted) && qmm_ts_supported(dn));
   ug.bm = dn.bm = pl.bm;
   ug.max_tiles = dn.max_tiles = max_tiles_for(R, E, pl.bm);
 
@@ -485,6 +501,10 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
     if (launch_gather_rows(x, rb.src_row, R, H, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
     ug.x = x_sorted;
     ug.src_row = nullptr;
+    if (pl.ts) {
+      if (launch_qmm_ts(ug, s) != cudaSuccess) return QMOE_ERR_CUDA;
+      return cuda_status(launch_qmm_ts(dn, s));
+    }
     if (launch_qmm_tc(ug, s) != cudaSuccess) return QMOE_ERR_CUDA;
     return cuda_status(launch_qmm_tc(dn, s));
   }

@@ -176,18 +176,23 @@ __device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
 }
 
 // --------------------------------------------------------------------- barriers
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+// Named barrier ID (an immediate, so the compiler sees every barrier a kernel uses).
+template <int ID>
+__device__ __forceinline__ void named_bar_sync(int nthreads) {
+  static_assert(ID > 0 && ID < 16, "named barrier id");
+  asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(nthreads) : "memory");
 }
 // Named barrier that also returns, to every participant, whether any of them passed
 // `pred` true: a decision all of them take together.
-__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+template <int ID>
+__device__ __forceinline__ bool named_bar_any(int nthreads, bool pred) {
+  static_assert(ID > 0 && ID < 16, "named barrier id");
   uint32_t r;
   asm volatile(
       "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n"
       " selp.u32 %0, 1, 0, q;\n}"
       : "=r"(r)
-      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "r"(pred ? 1u : 0u), "n"(ID), "r"(nthreads)
       : "memory");
   return r != 0;
 }

@@ -127,6 +127,11 @@ bool qdec_supported(const GemmArgs& a);
 cudaError_t launch_qdec(const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream); // tiles of 128 rows
 bool qmm_tc_supported(const GemmArgs& a);
+// Tensor-core kernel with the dequantised weights as the MMA A operand in tensor memory,
+// for tiles of up to kTsTileRows rows: 4-bit codes, activations already in tile order.
+constexpr int kTsTileRows = 192;
+bool qmm_ts_supported(const GemmArgs& a);
+cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream);
 
 // ------------------------------------------------------------------------ combine
 cudaError_t launch_combine(const uint16_t* y_sorted, const uint32_t* inv_order,

@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) qdec_kernel(const __grid_constant
       const uint32_t buf = tc & 1;
       bool stop = *abort_flag || !mbar_wait(&d_full[buf], (tc >> 1) & 1, p.d_status);
       // the SwitchGLU path meets at a named barrier below: its warps stop together
-      if (!p.pair) stop = named_bar_any(1, kEpiWarps * 32, stop);
+      if (!p.pair) stop = named_bar_any<1>(kEpiWarps * 32, stop);
       if (stop) { *abort_flag = 1; break; }
       tc_fence_after();
       float v[kNt];
@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) qdec_kernel(const __grid_constant
 #pragma unroll
           for (int t = 0; t < kNt; ++t) xchg[(r - 64) * kXchgStride + t] = v[t];
         }
-        named_bar_sync(1, kEpiWarps * 32);
+        named_bar_sync<1>(kEpiWarps * 32);
         if (r < 64 && n0 + r < p.N) {
 #pragma unroll
           for (int t = 0; t < kNt; ++t) {
@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) qdec_kernel(const __grid_constant
             }
           }
         }
-        named_bar_sync(1, kEpiWarps * 32);  // before the next unit overwrites xchg
+        named_bar_sync<1>(kEpiWarps * 32);  // before the next unit overwrites xchg
       } else if (n0 + r < p.N) {
 #pragma unroll
         for (int t = 0; t < kNt; ++t) {

@@ -1,0 +1,563 @@
+// Tensor-core gathered quantised matmul for many rows per expert (prefill), with the
+// dequantised weights as the MMA's A operand in tensor memory.
+//
+// The product of the other two kernels -- for every expert-aligned tile of routed rows
+// (MLX PR #4567 "[Metal] Gather mm improvement", Proposed changes) and every block of
+// output channels, y[row, n] = x[row] . dequantize(W[e])[n]^T (nuvec-core 0.4.0
+// tests/quantized.rs, gather_qmm_selects_batches), with the SwitchGLU epilogue
+// h = silu(gate) * up for two weight stacks (MLX issue #4509 repro script, `moe`).
+//
+// Roles are those of a weight-stationary tile: a unit is 128 weight rows (64 channels of
+// both stacks, or 128 channels of one) against one tile of up to 192 routed rows of one
+// expert.  The weight rows are dequantised (q*s + b, one bf16 rounding) straight into
+// tensor memory as the M = 128 A operand; the tile's rows are the N operand, read by the
+// MMA from 128B-swizzled shared memory; N is the tile's valid row count rounded up to
+// 16, so a sparsely routed expert costs MMA work in proportion to its rows.  Against a
+// kernel that stages dequantised weights in shared memory, this halves the
+// dequantisation per flop (128 weight rows per 192 routed rows instead of 256 per 128)
+// and takes the weight tiles out of shared memory, whose bandwidth the MMAs' operand
+// reads, the activation copies and the weight stores otherwise exceed.
+//
+// One persistent CTA per SM takes every gridDim-th unit.  Warps:
+//   0-3, 15-18  epilogue, two groups taking alternate pieces: tcgen05.ld of the unit's
+//         128 x N fp32 accumulator in 32-column pieces (one TMEM lane per weight row),
+//         transposed through shared memory into 16-byte stores of 8 output channels
+//         (after silu*mul for two stacks) per valid routed row;
+//   4     activation producer: TMA of the activation slab of each 64-k step (one box of
+//         64, 128 or 192 rows x 128 B: as many rows as the tile's MMA N reads);
+//   5     MMA issuer: tcgen05.mma kind::f16, A from tensor memory, M=128, N <= 192, K=16;
+//   6-13  dequant: warp w owns the weight rows of TMEM lane quarter w%4 and one half of
+//         each step's 64 k (four packed words per thread and step);
+//   14    weight producer: TMA of the packed codes every 256 k (two boxes of 64 rows x
+//         128 B) and of the scales and biases every 8 groups.
+// Tensor memory: four 64-k A slots (128 columns) and two 192-column accumulators.
+// Every mbarrier wait is bounded; a timeout sets QMOE_DEV_TIMEOUT, stops all roles,
+// drains the copies and MMAs in flight and frees the tensor memory.
+#include <algorithm>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "qmoe_common.cuh"
+#include "qmoe_internal.h"
+#include "qmoe_tcgen05.cuh"
+#include "qmoe_tma.h"
+
+namespace qmoe {
+namespace {
+
+constexpr int kM = 128;                          // weight rows per unit = TMEM lanes = MMA M
+constexpr int kNMax = kTsTileRows;               // routed rows per tile: MMA N at most
+constexpr int kKC = 64;                          // k per step: one 128-byte bf16 row of the slab
+constexpr int kXBoxRows = 64;                    // activation rows per TMA box
+constexpr int kXBoxBytes = kXBoxRows * kKC * 2;  // 8 KB
+constexpr int kXBytes = kNMax * kKC * 2;         // 24 KB per activation stage
+constexpr int kS1 = 6;                           // activation stages
+constexpr int kPK = 4;                           // steps per packed-code slot (256 k)
+constexpr int kPBytes = kM * 128;                // 16 KB: two boxes of 64 rows x 128 B
+constexpr int kSP = 2;                           // packed-code slots
+constexpr int kSbGroups = 8;                     // groups per scale/bias box
+constexpr int kSbBytes = 2 * 2 * 64 * kSbGroups * 2;  // [box][s|b][64 rows][8] bf16
+constexpr int kSbSlots = 2;
+constexpr int kASlots = 4;                       // dequantised A tiles in tensor memory
+constexpr int kACols = kKC / 2;                  // TMEM columns per A tile (bf16 pairs)
+constexpr int kDCol0 = kASlots * kACols;         // accumulators after the A tiles
+constexpr int kTmemCols = 512;
+constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps = 8;
+constexpr int kProdWWarp = kDqWarp0 + kDqWarps;       // 14: packed codes, scales, biases
+constexpr int kEpi2Warp0 = kProdWWarp + 1;            // 15-18: second epilogue group
+constexpr int kThreads = (kEpi2Warp0 + kEpiWarps) * 32;  // 608
+constexpr int kEpiCols = 32;                     // accumulator columns (routed rows) per piece
+constexpr int kOffP = kS1 * kXBytes;
+constexpr int kOffSb = kOffP + kSP * kPBytes;
+constexpr int kStageBytes = kEpiCols * kM * 4;           // epilogue transpose: [32 rows][128] f32
+constexpr int kOffStage = kOffSb + kSbSlots * kSbBytes;  // one per epilogue group
+constexpr int kOffBar = kOffStage + 2 * kStageBytes;
+constexpr int kSmem = kOffBar + 512;
+static_assert(kDCol0 + 2 * kNMax <= kTmemCols, "tensor memory budget");
+static_assert(kSmem + 1024 <= 227 * 1024, "shared memory budget");
+static_assert(kXBytes % 1024 == 0 && kOffP % 1024 == 0 && kOffSb % 1024 == 0,
+              "128B-swizzled boxes need 1 KB alignment");
+static_assert(kNMax % kXBoxRows == 0 && kNMax % 16 == 0 && kNMax <= 256, "tile rows");
+
+// Instruction descriptor without N: fp32 accumulator, bf16 A and B, both K-major, M=128.
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kM >> 4) << 24);
+
+struct alignas(64) TsParams {
+  CUtensorMap tm_w[2];      // packed codes [E*N, K/8] u32, box {32 words, 64 rows}, 128B swizzle
+  CUtensorMap tm_sb[2][2];  // [stack][scales|biases] [E*N, K/group] bf16, box {8, 64}
+  CUtensorMap tm_x[3];      // activation rows [x_rows, K] bf16, box {64, 64*(i+1)}, 128B swizzle
+  uint16_t* y;
+  const uint32_t* dst_row;
+  const uint32_t* tiles;
+  const uint32_t* num_tiles;
+  int64_t dense_rows;
+  int64_t N, K;
+  int pair;                 // 1: one stack, a unit is 128 of its channels
+  int vec_store;            // y rows start 16-byte aligned: 8 channels per store
+  int* d_status;
+  ProfSlot* prof;
+};
+
+struct TsTile {
+  uint32_t row_start, expert, valid;
+};
+
+__device__ __forceinline__ TsTile ts_tile(const TsParams& p, int64_t j) {
+  TsTile t;
+  if (p.dense_rows > 0) {
+    t.row_start = static_cast<uint32_t>(j * kNMax);
+    t.expert = 0;
+    t.valid = static_cast<uint32_t>(imin64(kNMax, p.dense_rows - j * kNMax));
+  } else {
+    t.row_start = p.tiles[3 * j];
+    t.expert = p.tiles[3 * j + 1];
+    t.valid = min(p.tiles[3 * j + 2], static_cast<uint32_t>(kNMax));
+  }
+  return t;
+}
+
+// MMA N for a tile: its valid rows rounded up to 16 (at least 16).
+__device__ __forceinline__ uint32_t ts_mma_n(uint32_t valid) {
+  return max(16u, (valid + 15u) & ~15u);
+}
+
+// One bf16 value in both halves of a bf16x2.
+__device__ __forceinline__ __nv_bfloat162 bcast_bf16(uint16_t v) {
+  const uint32_t b = static_cast<uint32_t>(v) * 0x10001u;
+  return *reinterpret_cast<const __nv_bfloat162*>(&b);
+}
+
+template <int GS>
+__global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_constant__ TsParams p) {
+  constexpr int KS_SB = kSbGroups * GS / kKC;  // steps per scale/bias window
+  static_assert((kSbGroups * GS) % kKC == 0 && KS_SB >= 1, "group size");
+  static_assert(GS >= kKC / 2, "a thread's 32 k lie in one group");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full1 = bars;                   // [kS1] TMA tx: activation slab
+  uint64_t* empty1 = full1 + kS1;           // [kS1] MMA commit
+  uint64_t* fullP = empty1 + kS1;           // [kSP] TMA tx: packed codes
+  uint64_t* emptyP = fullP + kSP;           // [kSP] dequant warps
+  uint64_t* full_sb = emptyP + kSP;         // [kSbSlots] TMA tx
+  uint64_t* empty_sb = full_sb + kSbSlots;  // [kSbSlots] dequant warps
+  uint64_t* a_full = empty_sb + kSbSlots;   // [kASlots] dequant warps: A tile written
+  uint64_t* a_empty = a_full + kASlots;     // [kASlots] MMA commit: A tile read
+  uint64_t* d_full = a_empty + kASlots;     // [2] MMA commit: accumulator ready
+  uint64_t* d_empty = d_full + 2;           // [2] epilogue warps: accumulator drained
+  uint64_t* drain = d_empty + 2;            // [1] final MMA commit on the abort path
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kS1; ++s) {
+      mbar_init(&full1[s], 1);
+      mbar_init(&empty1[s], 1);
+    }
+    for (int s = 0; s < kSP; ++s) {
+      mbar_init(&fullP[s], 1);
+      mbar_init(&emptyP[s], kDqWarps);
+    }
+    for (int s = 0; s < kSbSlots; ++s) {
+      mbar_init(&full_sb[s], 1);
+      mbar_init(&empty_sb[s], kDqWarps);
+    }
+    for (int s = 0; s < kASlots; ++s) {
+      mbar_init(&a_full[s], kDqWarps);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&d_full[s], 1);
+      mbar_init(&d_empty[s], 2 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_sh;
+  // inputs (tile table, activations) may come from the kernel before this one
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) prof_start(p.prof);
+
+  const int64_t KS = p.K / kKC;               // steps per unit
+  const int unit_n = p.pair ? kM : kM / 2;    // output channels per unit
+  const int64_t NB = (p.N + unit_n - 1) / unit_n;
+  const int64_t ntiles = p.dense_rows > 0 ? (p.dense_rows + kNMax - 1) / kNMax : *p.num_tiles;
+  const int64_t units = ntiles * NB;
+  // Units are dealt round-robin: the CTAs working on one tile's channel blocks at the same
+  // time share its activation rows through L2 (a tile is re-read once per channel block).
+  const int64_t u_begin = blockIdx.x, u_step = gridDim.x, u_end = units;
+  // first weight row of code box m (rows 0..63 and 64..127 of the unit)
+  auto box_row = [&](const TsTile& t, int64_t u, int m) -> int64_t {
+    const int64_t n0 = (u % NB) * unit_n;
+    return static_cast<int64_t>(t.expert) * p.N + n0 + (p.pair ? 64 * m : 0);
+  };
+
+  if (warp == kProdWarp) {
+    // ------------------------------------------------------- activation producer
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < 3; ++i) tma_prefetch_desc(&p.tm_x[i]);
+      uint32_t it = 0;
+      bool ab = false;
+      int64_t cur = -1;
+      TsTile tl{};
+      int nbox = 1;
+      for (int64_t u = u_begin; u < u_end && !ab; u += u_step) {
+        if (u / NB != cur) {
+          cur = u / NB;
+          tl = ts_tile(p, cur);
+          nbox = static_cast<int>((ts_mma_n(tl.valid) + kXBoxRows - 1) / kXBoxRows);
+        }
+        for (int64_t ks = 0; ks < KS; ++ks, ++it) {
+          if (*abort_flag) { ab = true; break; }
+          const uint32_t s1 = it % kS1;
+          if (!mbar_wait(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+          // one box of 64, 128 or 192 rows: as many as the tile's MMA N reads
+          mbar_arrive_expect_tx(&full1[s1], static_cast<uint32_t>(nbox * kXBoxBytes));
+          tma_load_2d(smem + s1 * kXBytes, &p.tm_x[nbox - 1], &full1[s1],
+                      static_cast<int32_t>(ks * kKC), static_cast<int32_t>(tl.row_start));
+        }
+      }
+      if (ab) {
+        // let the copies already issued land before the CTA can exit
+        const uint32_t f1 = it > static_cast<uint32_t>(kS1) ? it - kS1 : 0u;
+        for (uint32_t k = f1; k < it; ++k) mbar_wait(&full1[k % kS1], (k / kS1) & 1, nullptr);
+      }
+    }
+  } else if (warp == kProdWWarp) {
+    // ----------------------------------------------------------- weight producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_w[0]);
+      tma_prefetch_desc(&p.tm_w[1]);
+      uint32_t pbit = 0, sbit = 0;
+      bool ab = false;
+      int64_t cur = -1;
+      TsTile tl{};
+      for (int64_t u = u_begin; u < u_end && !ab; u += u_step) {
+        if (u / NB != cur) {
+          cur = u / NB;
+          tl = ts_tile(p, cur);
+        }
+        const int64_t r0 = box_row(tl, u, 0), r1 = box_row(tl, u, 1);
+        for (int64_t ks = 0; ks < KS; ++ks) {
+          if (*abort_flag) { ab = true; break; }
+          if (ks % kPK == 0) {
+            const uint32_t sp = pbit % kSP;
+            if (!mbar_wait(&emptyP[sp], ((pbit / kSP) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+            mbar_arrive_expect_tx(&fullP[sp], kPBytes);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+              tma_load_2d(smem + kOffP + sp * kPBytes + m * 64 * 128, &p.tm_w[m], &fullP[sp],
+                          static_cast<int32_t>((ks / kPK) * 32), static_cast<int32_t>(m ? r1 : r0));
+            ++pbit;
+          }
+          if (ks % KS_SB == 0) {
+            const uint32_t e = sbit % kSbSlots;
+            if (!mbar_wait(&empty_sb[e], ((sbit / kSbSlots) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+            mbar_arrive_expect_tx(&full_sb[e], kSbBytes);
+            const int32_t gx = static_cast<int32_t>(ks * kKC / GS);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+              for (int arr = 0; arr < 2; ++arr)
+                tma_load_2d(smem + kOffSb + e * kSbBytes + (m * 2 + arr) * 64 * kSbGroups * 2,
+                            &p.tm_sb[m][arr], &full_sb[e], gx, static_cast<int32_t>(m ? r1 : r0));
+            ++sbit;
+          }
+        }
+      }
+      if (ab) {
+        const uint32_t fp = pbit > static_cast<uint32_t>(kSP) ? pbit - kSP : 0u;
+        for (uint32_t k = fp; k < pbit; ++k) mbar_wait(&fullP[k % kSP], (k / kSP) & 1, nullptr);
+        const uint32_t fs = sbit > static_cast<uint32_t>(kSbSlots) ? sbit - kSbSlots : 0u;
+        for (uint32_t k = fs; k < sbit; ++k) mbar_wait(&full_sb[k % kSbSlots], (k / kSbSlots) & 1, nullptr);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------------- MMA issuer
+    // The whole warp walks the loop, so that addresses and descriptors stay
+    // warp-uniform; lane 0 waits and one elected lane (the same one throughout)
+    // issues the MMAs and the commits that track them.
+    uint32_t it = 0, tc = 0;
+    bool issued = false;
+    int ok = 1;
+    int64_t cur = -1;
+    uint32_t idesc = 0;
+    for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
+      if (u / NB != cur) {
+        cur = u / NB;
+        idesc = kIdescBase | ((ts_mma_n(ts_tile(p, cur).valid) >> 3) << 17);
+      }
+      const uint32_t buf = tc & 1;
+      if (lane == 0) ok = !*abort_flag && mbar_wait(&d_empty[buf], ((tc >> 1) & 1) ^ 1, p.d_status);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d = tmem_base + kDCol0 + buf * kNMax;
+      for (int64_t ks = 0; ks < KS; ++ks, ++it) {
+        const uint32_t s1 = it % kS1, as = it % kASlots;
+        if (lane == 0)
+          ok = mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) &&
+               mbar_wait(&a_full[as], (it / kASlots) & 1, p.d_status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t b0 = sw128_desc(smem + s1 * kXBytes);
+        const uint32_t a0 = tmem_base + as * kACols;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kKC / 16; ++kk)  // 32 bytes along k per step inside the atom
+            tc_mma_ts(d, a0 + kk * 8, b0 + 2 * kk, idesc, (ks | kk) != 0 ? 1u : 0u);
+          tc_commit(&empty1[s1]);
+          tc_commit(&a_empty[as]);
+        }
+        __syncwarp();
+        issued = true;
+      }
+      if (!ok) break;
+      if (elect_one()) tc_commit(&d_full[buf]);
+      __syncwarp();
+    }
+    __syncwarp();
+    const bool leader = elect_one();
+    if (leader && issued && *abort_flag) {
+      tc_commit(drain);  // completes when every MMA issued so far has finished
+      mbar_wait(drain, 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kDqWarps) {
+    // ------------------------------------------------------------------- dequant
+    // Warp w may only reach TMEM lanes 32*(w%4)..+31: it owns those weight rows, and
+    // half `part` of each step's 64 k (four packed words).
+    const int quarter = warp % 4, part = (warp - kDqWarp0) / 4;
+    const int r = quarter * 32 + lane;   // weight row of the unit = TMEM lane
+    const int m = r / 64, rr = r % 64;   // code box and row inside it
+    uint32_t it = 0, pbit = 0, sbit = 0;
+    for (int64_t u = u_begin; u < u_end; u += u_step) {
+      for (int64_t ks = 0; ks < KS; ++ks, ++it) {
+        if (*abort_flag) break;
+        const uint32_t sp = pbit % kSP, e = sbit % kSbSlots, as = it % kASlots;
+        if (ks % kPK == 0 && !mbar_wait(&fullP[sp], (pbit / kSP) & 1, p.d_status)) { *abort_flag = 1; break; }
+        if (ks % KS_SB == 0 &&
+            !mbar_wait(&full_sb[e], (sbit / kSbSlots) & 1, p.d_status)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&a_empty[as], ((it / kASlots) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        // this thread's 16 bytes of the row: piece (ks % 4)*2 + part of 8, at piece ^ (rr & 7)
+        const uint8_t* rowp = smem + kOffP + sp * kPBytes + m * 64 * 128 + rr * 128;
+        const int piece = static_cast<int>(ks % kPK) * 2 + part;
+        const uint4 pw = *reinterpret_cast<const uint4*>(rowp + ((piece ^ (rr & 7)) << 4));
+        // the group of these 32 k inside the scale window
+        const int g = (static_cast<int>((ks * kKC) % (kSbGroups * GS)) + part * (kKC / 2)) / GS;
+        const uint16_t* sbw = reinterpret_cast<const uint16_t*>(smem + kOffSb + e * kSbBytes);
+        const __nv_bfloat162 s2 = bcast_bf16(sbw[(m * 2 * 64 + rr) * kSbGroups + g]);
+        const __nv_bfloat162 b2 = bcast_bf16(sbw[((m * 2 + 1) * 64 + rr) * kSbGroups + g]);
+        const uint32_t w4[4] = {pw.x, pw.y, pw.z, pw.w};
+        uint32_t out[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 v = dequant_word4(w4[j], s2, b2);
+          out[4 * j + 0] = v.x;
+          out[4 * j + 1] = v.y;
+          out[4 * j + 2] = v.z;
+          out[4 * j + 3] = v.w;
+        }
+        // A tile: lane r, columns part*16.. (two bf16 of consecutive k per column)
+        tmem_st16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + as * kACols + part * 16, out);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        const bool p_done = ks % kPK == kPK - 1 || ks == KS - 1;
+        const bool sb_done = ks % KS_SB == KS_SB - 1 || ks == KS - 1;
+        if (lane == 0) {
+          mbar_arrive(&a_full[as]);
+          if (p_done) mbar_arrive(&emptyP[sp]);
+          if (sb_done) mbar_arrive(&empty_sb[e]);
+        }
+        if (p_done) ++pbit;
+        if (sb_done) ++sbit;
+      }
+      if (*abort_flag) break;
+    }
+  } else if (warp < kEpiWarps || warp >= kEpi2Warp0) {
+    // ------------------------------------------------------------------ epilogue
+    // Two groups of four warps take alternate pieces of 32 routed rows.  Per piece, each
+    // thread moves its TMEM lane (one weight row) into its group's [row][weight row] fp32
+    // stage; then the group's 128 threads take (routed row, 8 output channels) items,
+    // apply silu(gate)*up for two stacks (gate rows sit 64 after their up rows) and write
+    // 8 bf16 with one 16-byte store along the output row.
+    const int grp = warp < kEpiWarps ? 0 : 1;
+    const int quarter = warp % 4;        // a warp reaches TMEM lanes 32*(warp%4)..+31
+    const int r = quarter * 32 + lane;   // TMEM lane = weight row of the unit
+    // named barriers 1 and 2 (0 is __syncthreads), ids fixed at compile time
+    auto group_sync = [&]() {
+      if (grp == 0) named_bar_sync<1>(kEpiWarps * 32);
+      else named_bar_sync<2>(kEpiWarps * 32);
+    };
+    auto group_any = [&](bool pred) -> bool {
+      return grp == 0 ? named_bar_any<1>(kEpiWarps * 32, pred) : named_bar_any<2>(kEpiWarps * 32, pred);
+    };
+    float* stage = reinterpret_cast<float*>(smem + kOffStage + grp * kStageBytes);
+    const int nch = p.pair ? kM : kM / 2;  // output channels of a unit
+    const int groups = nch / 8;
+    uint32_t tc = 0;
+    int64_t cur = -1;
+    TsTile tl{};
+    for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
+      const uint32_t buf = tc & 1;
+      bool stop = *abort_flag || !mbar_wait(&d_full[buf], (tc >> 1) & 1, p.d_status);
+      stop = group_any(stop);  // the group meets at named barriers below
+      if (stop) { *abort_flag = 1; break; }
+      tc_fence_after();
+      if (u / NB != cur) {
+        cur = u / NB;
+        tl = ts_tile(p, cur);
+      }
+      const int64_t n0 = (u % NB) * unit_n;
+      const int pieces = static_cast<int>((ts_mma_n(tl.valid) + kEpiCols - 1) / kEpiCols);
+      if (grp >= pieces) {  // nothing for this group in this unit
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[buf]);
+        continue;
+      }
+      for (int pc = grp; pc < pieces; pc += 2) {
+        float v[kEpiCols];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kDCol0 + buf * kNMax +
+                      pc * kEpiCols, v);
+        if (pc + 2 >= pieces) {  // this group's last piece: its share of the accumulator is read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&d_empty[buf]);
+        }
+#pragma unroll
+        for (int j = 0; j < kEpiCols; ++j) stage[j * kM + r] = v[j];
+        group_sync();
+        const int t0 = pc * kEpiCols;
+        for (int item = r; item < kEpiCols * groups; item += kEpiWarps * 32) {
+          const int t = item / groups, c0 = (item % groups) * 8;
+          if (static_cast<uint32_t>(t0 + t) >= tl.valid) continue;
+          const float* srow = stage + t * kM;
+          float o[8];
+          const float4 a = *reinterpret_cast<const float4*>(srow + c0);
+          const float4 b = *reinterpret_cast<const float4*>(srow + c0 + 4);
+          o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+          o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+          if (!p.pair) {
+            const float4 ga = *reinterpret_cast<const float4*>(srow + 64 + c0);
+            const float4 gb = *reinterpret_cast<const float4*>(srow + 64 + c0 + 4);
+            const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] *= g[i] / (1.0f + expf(-g[i]));
+          }
+          const uint32_t pos = tl.row_start + t0 + t;
+          const uint32_t dr = p.dst_row ? p.dst_row[pos] : pos;
+          uint16_t* dst = p.y + static_cast<int64_t>(dr) * p.N + n0 + c0;
+          if (p.vec_store && n0 + c0 + 8 <= p.N) {
+            uint4 pk;
+            pk.x = f32_to_bf16(o[0]) | (static_cast<uint32_t>(f32_to_bf16(o[1])) << 16);
+            pk.y = f32_to_bf16(o[2]) | (static_cast<uint32_t>(f32_to_bf16(o[3])) << 16);
+            pk.z = f32_to_bf16(o[4]) | (static_cast<uint32_t>(f32_to_bf16(o[5])) << 16);
+            pk.w = f32_to_bf16(o[6]) | (static_cast<uint32_t>(f32_to_bf16(o[7])) << 16);
+            *reinterpret_cast<uint4*>(dst) = pk;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (n0 + c0 + i < p.N) dst[i] = f32_to_bf16(o[i]);
+          }
+        }
+        group_sync();  // before the next piece overwrites the stage
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+  if (threadIdx.x == 0) prof_end(p.prof);
+}
+
+template <int GS>
+cudaError_t launch_ts_gs(const TsParams& prm, cudaStream_t stream) {
+  auto kern = qmm_ts_kernel<GS>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem + 1024);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  LaunchTimer timer(prm.pair ? "ts" : "ts_glu", stream);
+  TsParams p = prm;
+  p.prof = timer.slot();
+  const cudaError_t e = launch_pdl(kern, dim3(sm_count()), dim3(kThreads), kSmem + 1024, stream, p);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool qmm_ts_supported(const GemmArgs& a) {
+  if (a.bits != 4 || (a.group != 32 && a.group != 64 && a.group != 128)) return false;
+  if (a.K % kKC != 0) return false;                    // whole 64-k activation boxes
+  if ((a.K / a.group) % kSbGroups != 0) return false;  // scale/bias rows: 16-byte pitch
+  if (a.x_rows <= 0 || a.src_row != nullptr) return false;  // activations in tile order
+  return true;
+}
+
+cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream) {
+  if (!qmm_ts_supported(a)) return cudaErrorNotSupported;
+  if (a.dense_rows <= 0 && a.bm != kNMax) return cudaErrorInvalidValue;  // tile table of kNMax rows
+  TsParams prm{};
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < 3; ++i) {
+    e = make_tmap_2d_bf16(&prm.tm_x[i], a.x, a.K, a.x_rows, kKC, kXBoxRows * (i + 1),
+                          /*swizzle128=*/true);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t words = a.K / 8;
+  const int64_t gpr = a.K / a.group;
+  for (int m = 0; m < 2; ++m) {
+    const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
+    e = make_tmap_2d_u32(&prm.tm_w[m], wm.codes, words, a.E * a.N, 32, 64, /*swizzle128=*/true);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d_bf16(&prm.tm_sb[m][0], wm.scales, gpr, a.E * a.N, kSbGroups, 64, false);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d_bf16(&prm.tm_sb[m][1], wm.biases, gpr, a.E * a.N, kSbGroups, 64, false);
+    if (e != cudaSuccess) return e;
+  }
+  prm.y = a.y;
+  prm.dst_row = a.dst_row;
+  prm.tiles = a.tiles;
+  prm.num_tiles = a.num_tiles;
+  prm.dense_rows = a.dense_rows;
+  prm.N = a.N;
+  prm.K = a.K;
+  prm.pair = a.nmat == 2 ? 0 : 1;
+  prm.vec_store = (a.N % 8 == 0 && reinterpret_cast<uintptr_t>(a.y) % 16 == 0) ? 1 : 0;
+  prm.d_status = a.d_status;
+  if (a.group == 32) return launch_ts_gs<32>(prm, stream);
+  if (a.group == 64) return launch_ts_gs<64>(prm, stream);
+  return launch_ts_gs<128>(prm, stream);
+}
+
+}  // namespace qmoe

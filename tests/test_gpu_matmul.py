@@ -22,17 +22,22 @@ from inputs import (bf16_bits, decode_tokens, decode_weights, dense_projections,
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["qmv", "qdec", "tc", "auto"])
+@pytest.fixture(params=["qmv", "qdec", "tc", "tc_smem", "auto"])
 def kernel(request, monkeypatch):
     """Kernel choice: forced streaming (mma.sync, or tcgen05 where it supports the shape),
-    forced tensor-core tiles, or the library's own plan (chosen from the most rows one
-    expert can receive)."""
+    forced tensor-core tiles (weights in tensor memory where the shape allows, or staged
+    in shared memory), or the library's own plan (chosen from the most rows one expert
+    can receive)."""
     monkeypatch.delenv("QMOE_DECODE", raising=False)
+    monkeypatch.delenv("QMOE_PREFILL", raising=False)
     if request.param == "auto":
         monkeypatch.delenv("QMOE_FORCE_KERNEL", raising=False)
     elif request.param == "qdec":
         monkeypatch.setenv("QMOE_FORCE_KERNEL", "qmv")
         monkeypatch.setenv("QMOE_DECODE", "qdec")
+    elif request.param == "tc_smem":
+        monkeypatch.setenv("QMOE_FORCE_KERNEL", "tc")
+        monkeypatch.setenv("QMOE_PREFILL", "tc")
     else:
         monkeypatch.setenv("QMOE_FORCE_KERNEL", request.param)
     return request.param
