@@ -51,10 +51,19 @@ constexpr int kKC = 64;                          // k per step: one 128-byte bf1
 constexpr int kXBoxRows = 64;                    // activation rows per TMA box
 constexpr int kXBoxBytes = kXBoxRows * kKC * 2;  // 8 KB
 constexpr int kXBytes = kNMax * kKC * 2;         // 24 KB per activation stage
-constexpr int kS1 = 6;                           // activation stages
+#ifndef QTS_S1
+#define QTS_S1 6
+#endif
+#ifndef QTS_SP
+#define QTS_SP 2
+#endif
+#ifndef QTS_EPI_COLS
+#define QTS_EPI_COLS 32
+#endif
+constexpr int kS1 = QTS_S1;                      // activation stages
 constexpr int kPK = 4;                           // steps per packed-code slot (256 k)
 constexpr int kPBytes = kM * 128;                // 16 KB: two boxes of 64 rows x 128 B
-constexpr int kSP = 2;                           // packed-code slots
+constexpr int kSP = QTS_SP;                      // packed-code slots
 constexpr int kSbGroups = 8;                     // groups per scale/bias box
 constexpr int kSbBytes = 2 * 2 * 64 * kSbGroups * 2;  // [box][s|b][64 rows][8] bf16
 constexpr int kSbSlots = 2;
@@ -66,10 +75,11 @@ constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps
 constexpr int kProdWWarp = kDqWarp0 + kDqWarps;       // 14: packed codes, scales, biases
 constexpr int kEpi2Warp0 = kProdWWarp + 1;            // 15-18: second epilogue group
 constexpr int kThreads = (kEpi2Warp0 + kEpiWarps) * 32;  // 608
-constexpr int kEpiCols = 32;                     // accumulator columns (routed rows) per piece
+constexpr int kEpiCols = QTS_EPI_COLS;           // accumulator columns (routed rows) per piece
+static_assert(kEpiCols == 16 || kEpiCols == 32, "epilogue piece");
 constexpr int kOffP = kS1 * kXBytes;
 constexpr int kOffSb = kOffP + kSP * kPBytes;
-constexpr int kStageBytes = kEpiCols * kM * 4;           // epilogue transpose: [32 rows][128] f32
+constexpr int kStageBytes = kEpiCols * kM * 4;           // epilogue transpose: [rows][128] f32
 constexpr int kOffStage = kOffSb + kSbSlots * kSbBytes;  // one per epilogue group
 constexpr int kOffBar = kOffStage + 2 * kStageBytes;
 constexpr int kSmem = kOffBar + 512;
@@ -120,6 +130,10 @@ __device__ __forceinline__ TsTile ts_tile(const TsParams& p, int64_t j) {
 __device__ __forceinline__ uint32_t ts_mma_n(uint32_t valid) {
   return max(16u, (valid + 15u) & ~15u);
 }
+
+// One epilogue piece of accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[32]) { tmem_ld32(taddr, v); }
+__device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
 
 // One bf16 value in both halves of a bf16x2.
 __device__ __forceinline__ __nv_bfloat162 bcast_bf16(uint16_t v) {
@@ -438,8 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
       }
       for (int pc = grp; pc < pieces; pc += 2) {
         float v[kEpiCols];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kDCol0 + buf * kNMax +
-                      pc * kEpiCols, v);
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kDCol0 +
+                               buf * kNMax + pc * kEpiCols;
+        tmem_ld_piece(taddr, v);
         if (pc + 2 >= pieces) {  // this group's last piece: its share of the accumulator is read
           tc_fence_before();
           __syncwarp();

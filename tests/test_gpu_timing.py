@@ -42,16 +42,22 @@ def test_timing_slots_eager_and_graph(gpu_lib):
 
 
 def test_forced_kernels_really_run(gpu_lib, monkeypatch):
-    """QMOE_FORCE_KERNEL selects the streaming or the tensor-core kernel: the launch
-    records prove which one ran (so the parity tests cover both)."""
+    """QMOE_FORCE_KERNEL selects the streaming or a tensor-core kernel (QMOE_PREFILL=tc
+    picks the one that stages weights in shared memory over the one that keeps them in
+    tensor memory): the launch records prove which one ran (so the parity tests cover
+    each)."""
     q = gpu_lib
     rng = np.random.default_rng(3)
     w, s, b = random_qweight(rng, 1, 256, 512, 64, 4)
     args = (dev_u32(w[0]), dev_bf16(s[0]), dev_bf16(b[0]), 64, 4)
     x = dev_bf16(normal_bf16(rng, (200, 512)))
     slots = torch.zeros(16 * 8, dtype=torch.uint8, device="cuda")
-    for forced, name in (("qmv", "qmv"), ("tc", "tc")):
+    for forced, prefill, name in (("qmv", None, "qmv"), ("tc", None, "ts"), ("tc", "tc", "tc")):
         monkeypatch.setenv("QMOE_FORCE_KERNEL", forced)
+        if prefill is None:
+            monkeypatch.delenv("QMOE_PREFILL", raising=False)
+        else:
+            monkeypatch.setenv("QMOE_PREFILL", prefill)
         q.qmoe_qmm(x, *args)  # warm-up outside timing
         torch.cuda.synchronize()
         q.qmoe_timing_enable(slots)
