@@ -23,14 +23,17 @@
 //         128 x N fp32 accumulator in 32-column pieces (one TMEM lane per weight row),
 //         transposed through shared memory into 16-byte stores of 8 output channels
 //         (after silu*mul for two stacks) per valid routed row;
-//   4     activation producer: TMA of the activation slab of each 64-k step (one box of
-//         64, 128 or 192 rows x 128 B: as many rows as the tile's MMA N reads);
+//   4     activation producer: TMA of the activation slab of each 128-k step (per 64-k
+//         swizzle atom one box of 64, 128 or 192 rows x 128 B: as many rows as the tile's
+//         MMA N reads);
 //   5     MMA issuer: tcgen05.mma kind::f16, A from tensor memory, M=128, N <= 192, K=16;
 //   6-13  dequant: warp w owns the weight rows of TMEM lane quarter w%4 and one half of
-//         each step's 64 k (four packed words per thread and step);
+//         each step's 128 k (eight packed words per thread and step);
 //   14    weight producer: TMA of the packed codes every 256 k (two boxes of 64 rows x
 //         128 B) and of the scales and biases every 8 groups.
-// Tensor memory: four 64-k A slots (128 columns) and two 192-column accumulators.
+// Tensor memory: two 128-k A slots (128 columns) and two 192-column accumulators.  Steps
+// of 128 k rather than 64 halve the mbarrier hand-offs between the roles per flop, which
+// bound the kernel (64-k steps: T=16384 up/gate 684 TFLOP/s; 128-k steps: 885).
 // Every mbarrier wait is bounded; a timeout sets QMOE_DEV_TIMEOUT, stops all roles,
 // drains the copies and MMAs in flight and frees the tensor memory.
 #include <algorithm>
@@ -47,12 +50,19 @@ namespace {
 
 constexpr int kM = 128;                          // weight rows per unit = TMEM lanes = MMA M
 constexpr int kNMax = kTsTileRows;               // routed rows per tile: MMA N at most
-constexpr int kKC = 64;                          // k per step: one 128-byte bf16 row of the slab
+#ifndef QTS_KC
+#define QTS_KC 128
+#endif
+constexpr int kAtomK = 64;                       // k per 128-byte swizzle atom of bf16
+constexpr int kKC = QTS_KC;                      // k per step
+constexpr int kAtoms = kKC / kAtomK;             // activation atoms per step
 constexpr int kXBoxRows = 64;                    // activation rows per TMA box
-constexpr int kXBoxBytes = kXBoxRows * kKC * 2;  // 8 KB
-constexpr int kXBytes = kNMax * kKC * 2;         // 24 KB per activation stage
+constexpr int kXBoxBytes = kXBoxRows * kAtomK * 2;  // 8 KB: 64 rows of one atom
+constexpr int kXAtomBytes = kNMax * kAtomK * 2;     // 24 KB: one atom of a full tile
+constexpr int kXBytes = kAtoms * kXAtomBytes;       // per activation stage
+static_assert(kKC == 64 || kKC == 128, "step");
 #ifndef QTS_S1
-#define QTS_S1 6
+#define QTS_S1 (6 / (QTS_KC / 64))
 #endif
 #ifndef QTS_SP
 #define QTS_SP 2
@@ -61,14 +71,15 @@ constexpr int kXBytes = kNMax * kKC * 2;         // 24 KB per activation stage
 #define QTS_EPI_COLS 32
 #endif
 constexpr int kS1 = QTS_S1;                      // activation stages
-constexpr int kPK = 4;                           // steps per packed-code slot (256 k)
+constexpr int kPK = 256 / kKC;                   // steps per packed-code slot (256 k)
 constexpr int kPBytes = kM * 128;                // 16 KB: two boxes of 64 rows x 128 B
 constexpr int kSP = QTS_SP;                      // packed-code slots
 constexpr int kSbGroups = 8;                     // groups per scale/bias box
 constexpr int kSbBytes = 2 * 2 * 64 * kSbGroups * 2;  // [box][s|b][64 rows][8] bf16
 constexpr int kSbSlots = 2;
-constexpr int kASlots = 4;                       // dequantised A tiles in tensor memory
 constexpr int kACols = kKC / 2;                  // TMEM columns per A tile (bf16 pairs)
+constexpr int kASlots = 128 / kACols;            // dequantised A tiles in tensor memory
+constexpr int kTW = kKC / 16;                    // packed words per dequant thread and step
 constexpr int kDCol0 = kASlots * kACols;         // accumulators after the A tiles
 constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps = 8;
@@ -131,6 +142,10 @@ __device__ __forceinline__ uint32_t ts_mma_n(uint32_t valid) {
   return max(16u, (valid + 15u) & ~15u);
 }
 
+// One dequantised A slice (16 or 32 columns) of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[16]) { tmem_st16(taddr, r); }
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st32(taddr, r); }
+
 // One epilogue piece of accumulator columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[32]) { tmem_ld32(taddr, v); }
 __device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
@@ -145,7 +160,7 @@ template <int GS>
 __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_constant__ TsParams p) {
   constexpr int KS_SB = kSbGroups * GS / kKC;  // steps per scale/bias window
   static_assert((kSbGroups * GS) % kKC == 0 && KS_SB >= 1, "group size");
-  static_assert(GS >= kKC / 2, "a thread's 32 k lie in one group");
+  constexpr int GPT = (kKC / 2) >= GS ? (kKC / 2) / GS : 1;  // groups of a thread's k per step
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -238,9 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
           const uint32_t s1 = it % kS1;
           if (!mbar_wait(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
           // one box of 64, 128 or 192 rows: as many as the tile's MMA N reads
-          mbar_arrive_expect_tx(&full1[s1], static_cast<uint32_t>(nbox * kXBoxBytes));
-          tma_load_2d(smem + s1 * kXBytes, &p.tm_x[nbox - 1], &full1[s1],
-                      static_cast<int32_t>(ks * kKC), static_cast<int32_t>(tl.row_start));
+          mbar_arrive_expect_tx(&full1[s1], static_cast<uint32_t>(kAtoms * nbox * kXBoxBytes));
+#pragma unroll
+          for (int a = 0; a < kAtoms; ++a)
+            tma_load_2d(smem + s1 * kXBytes + a * kXAtomBytes, &p.tm_x[nbox - 1], &full1[s1],
+                        static_cast<int32_t>(ks * kKC + a * kAtomK), static_cast<int32_t>(tl.row_start));
         }
       }
       if (ab) {
@@ -336,8 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
         const uint32_t a0 = tmem_base + as * kACols;
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kKC / 16; ++kk)  // 32 bytes along k per step inside the atom
-            tc_mma_ts(d, a0 + kk * 8, b0 + 2 * kk, idesc, (ks | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kKC / 16; ++kk)  // atom kk/4, 32 bytes along k inside it
+            tc_mma_ts(d, a0 + kk * 8, b0 + ((kk / 4) * kXAtomBytes >> 4) + 2 * (kk % 4), idesc,
+                      (ks | kk) != 0 ? 1u : 0u);
           tc_commit(&empty1[s1]);
           tc_commit(&a_empty[as]);
         }
@@ -358,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
   } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kDqWarps) {
     // ------------------------------------------------------------------- dequant
     // Warp w may only reach TMEM lanes 32*(w%4)..+31: it owns those weight rows, and
-    // half `part` of each step's 64 k (four packed words).
+    // half `part` of each step's k (kTW packed words).
     const int quarter = warp % 4, part = (warp - kDqWarp0) / 4;
     const int r = quarter * 32 + lane;   // weight row of the unit = TMEM lane
     const int m = r / 64, rr = r % 64;   // code box and row inside it
@@ -372,27 +390,34 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
             !mbar_wait(&full_sb[e], (sbit / kSbSlots) & 1, p.d_status)) { *abort_flag = 1; break; }
         if (!mbar_wait(&a_empty[as], ((it / kASlots) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
         tc_fence_after();
-        // this thread's 16 bytes of the row: piece (ks % 4)*2 + part of 8, at piece ^ (rr & 7)
+        // this thread's kTW words of the row: 16-byte pieces of the slot's 128-byte row,
+        // piece c at c ^ (rr & 7)
         const uint8_t* rowp = smem + kOffP + sp * kPBytes + m * 64 * 128 + rr * 128;
-        const int piece = static_cast<int>(ks % kPK) * 2 + part;
-        const uint4 pw = *reinterpret_cast<const uint4*>(rowp + ((piece ^ (rr & 7)) << 4));
-        // the group of these 32 k inside the scale window
-        const int g = (static_cast<int>((ks * kKC) % (kSbGroups * GS)) + part * (kKC / 2)) / GS;
+        // the thread's k lie in GPT groups, the first at g0 of the scale window
+        const int g0 = (static_cast<int>((ks * kKC) % (kSbGroups * GS)) + part * (kKC / 2)) / GS;
         const uint16_t* sbw = reinterpret_cast<const uint16_t*>(smem + kOffSb + e * kSbBytes);
-        const __nv_bfloat162 s2 = bcast_bf16(sbw[(m * 2 * 64 + rr) * kSbGroups + g]);
-        const __nv_bfloat162 b2 = bcast_bf16(sbw[((m * 2 + 1) * 64 + rr) * kSbGroups + g]);
-        const uint32_t w4[4] = {pw.x, pw.y, pw.z, pw.w};
-        uint32_t out[16];
+        __nv_bfloat162 s2[GPT], b2[GPT];
+        load_group_pairs<GPT>(sbw + (m * 2 * 64 + rr) * kSbGroups + g0, s2);
+        load_group_pairs<GPT>(sbw + ((m * 2 + 1) * 64 + rr) * kSbGroups + g0, b2);
+        uint32_t out[kTW * 4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 v = dequant_word4(w4[j], s2, b2);
-          out[4 * j + 0] = v.x;
-          out[4 * j + 1] = v.y;
-          out[4 * j + 2] = v.z;
-          out[4 * j + 3] = v.w;
+        for (int q = 0; q < kTW / 4; ++q) {
+          const int piece = static_cast<int>(ks % kPK) * (kKC / 32) + part * (kTW / 4) + q;
+          const uint4 pw = *reinterpret_cast<const uint4*>(rowp + ((piece ^ (rr & 7)) << 4));
+          const uint32_t w4[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int gi = ((4 * q + j) * 8) / GS;  // the word's group among the thread's
+            const uint4 v = dequant_word4(w4[j], s2[gi], b2[gi]);
+            out[(4 * q + j) * 4 + 0] = v.x;
+            out[(4 * q + j) * 4 + 1] = v.y;
+            out[(4 * q + j) * 4 + 2] = v.z;
+            out[(4 * q + j) * 4 + 3] = v.w;
+          }
         }
-        // A tile: lane r, columns part*16.. (two bf16 of consecutive k per column)
-        tmem_st16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + as * kACols + part * 16, out);
+        // A tile: lane r, columns part*kTW*4.. (two bf16 of consecutive k per column)
+        tmem_st_cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + as * kACols +
+                         part * (kTW * 4), out);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -533,7 +558,7 @@ cudaError_t launch_ts_gs(const TsParams& prm, cudaStream_t stream) {
 
 bool qmm_ts_supported(const GemmArgs& a) {
   if (a.bits != 4 || (a.group != 32 && a.group != 64 && a.group != 128)) return false;
-  if (a.K % kKC != 0) return false;                    // whole 64-k activation boxes
+  if (a.K % kKC != 0) return false;                    // whole steps of activation boxes
   if ((a.K / a.group) % kSbGroups != 0) return false;  // scale/bias rows: 16-byte pitch
   if (a.x_rows <= 0 || a.src_row != nullptr) return false;  // activations in tile order
   return true;
@@ -545,7 +570,7 @@ cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream) {
   TsParams prm{};
   cudaError_t e = cudaSuccess;
   for (int i = 0; i < 3; ++i) {
-    e = make_tmap_2d_bf16(&prm.tm_x[i], a.x, a.K, a.x_rows, kKC, kXBoxRows * (i + 1),
+    e = make_tmap_2d_bf16(&prm.tm_x[i], a.x, a.K, a.x_rows, kAtomK, kXBoxRows * (i + 1),
                           /*swizzle128=*/true);
     if (e != cudaSuccess) return e;
   }

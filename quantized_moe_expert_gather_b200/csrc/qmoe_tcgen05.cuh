@@ -149,4 +149,25 @@ __device__ __forceinline__ uint4 dequant_word4(uint32_t w, __nv_bfloat162 s2, __
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+// NG consecutive bf16 values (NG = 1, 2 or 4; p aligned to 2*NG bytes), each broadcast
+// to both halves of a bf16x2.
+template <int NG>
+__device__ __forceinline__ void load_group_pairs(const uint16_t* p, __nv_bfloat162 (&out)[NG]) {
+  uint32_t w[(NG + 1) / 2];
+  if constexpr (NG == 4) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else if constexpr (NG == 2) {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  } else {
+    w[0] = *p;
+  }
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    const uint32_t b = prmt(w[g / 2], 0u, (g & 1) ? 0x3232u : 0x1010u);
+    out[g] = *reinterpret_cast<const __nv_bfloat162*>(&b);
+  }
+}
+
 }  // namespace qmoe
