@@ -107,6 +107,7 @@ struct alignas(64) TsParams {
   CUtensorMap tm_w[2];      // packed codes [E*N, K/8] u32, box {32 words, 64 rows}, 128B swizzle
   CUtensorMap tm_sb[2][2];  // [stack][scales|biases] [E*N, K/group] bf16, box {8, 64}
   CUtensorMap tm_x[3];      // activation rows [x_rows, K] bf16, box {64, 64*(i+1)}, 128B swizzle
+  CUtensorMap tm_y;         // output rows [x_rows, N] bf16, box {128, kEpiCols} (tma_store only)
   uint16_t* y;
   const uint32_t* dst_row;
   const uint32_t* tiles;
@@ -115,6 +116,8 @@ struct alignas(64) TsParams {
   int64_t N, K;
   int pair;                 // 1: one stack, a unit is 128 of its channels
   int vec_store;            // y rows start 16-byte aligned: 8 channels per store
+  int tma_store;            // one stack, rows in tile order (no dst_row), vec_store: full
+                            // epilogue pieces leave by TMA tensor stores
   int* d_status;
   ProfSlot* prof;
 };
@@ -142,19 +145,6 @@ __device__ __forceinline__ uint32_t ts_mma_n(uint32_t valid) {
   return max(16u, (valid + 15u) & ~15u);
 }
 
-// One dequantised A slice (16 or 32 columns) of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[16]) { tmem_st16(taddr, r); }
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st32(taddr, r); }
-
-// One epilogue piece of accumulator columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[32]) { tmem_ld32(taddr, v); }
-__device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
-
-// One bf16 value in both halves of a bf16x2.
-__device__ __forceinline__ __nv_bfloat162 bcast_bf16(uint16_t v) {
-  const uint32_t b = static_cast<uint32_t>(v) * 0x10001u;
-  return *reinterpret_cast<const __nv_bfloat162*>(&b);
-}
 
 template <int GS>
 __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_constant__ TsParams p) {
@@ -485,10 +475,27 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
           __syncwarp();
           if (lane == 0) mbar_arrive(&d_empty[buf]);
         }
+        const int t0 = pc * kEpiCols;
+        // the stage is free once this group's previous tensor store has read it
+        if (r == 0 && p.tma_store) bulk_wait_read_all();
+        group_sync();
+        if (p.tma_store && static_cast<uint32_t>(t0 + kEpiCols) <= tl.valid) {
+          // a full piece of one stack in tile order: bf16 [rows][128 channels], one TMA store
+          uint16_t* sb16 = reinterpret_cast<uint16_t*>(stage);
+#pragma unroll
+          for (int j = 0; j < kEpiCols; ++j) sb16[j * kM + r] = f32_to_bf16(v[j]);
+          fence_proxy_async_smem();
+          group_sync();
+          if (r == 0) {
+            tma_store_2d(&p.tm_y, stage, static_cast<int32_t>(n0),
+                         static_cast<int32_t>(tl.row_start + t0));
+            bulk_commit_group();
+          }
+          continue;
+        }
 #pragma unroll
         for (int j = 0; j < kEpiCols; ++j) stage[j * kM + r] = v[j];
         group_sync();
-        const int t0 = pc * kEpiCols;
         for (int item = r; item < kEpiCols * groups; item += kEpiWarps * 32) {
           const int t = item / groups, c0 = (item % groups) * 8;
           if (static_cast<uint32_t>(t0 + t) >= tl.valid) continue;
@@ -509,11 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
           const uint32_t dr = p.dst_row ? p.dst_row[pos] : pos;
           uint16_t* dst = p.y + static_cast<int64_t>(dr) * p.N + n0 + c0;
           if (p.vec_store && n0 + c0 + 8 <= p.N) {
-            uint4 pk;
-            pk.x = f32_to_bf16(o[0]) | (static_cast<uint32_t>(f32_to_bf16(o[1])) << 16);
-            pk.y = f32_to_bf16(o[2]) | (static_cast<uint32_t>(f32_to_bf16(o[3])) << 16);
-            pk.z = f32_to_bf16(o[4]) | (static_cast<uint32_t>(f32_to_bf16(o[5])) << 16);
-            pk.w = f32_to_bf16(o[6]) | (static_cast<uint32_t>(f32_to_bf16(o[7])) << 16);
+            const uint4 pk = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                        pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
             *reinterpret_cast<uint4*>(dst) = pk;
           } else {
 #pragma unroll
@@ -521,9 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
               if (n0 + c0 + i < p.N) dst[i] = f32_to_bf16(o[i]);
           }
         }
-        group_sync();  // before the next piece overwrites the stage
       }
     }
+    if (r == 0 && p.tma_store) bulk_wait_all();  // the tensor stores have landed
   }
 
   // ------------------------------------------------------------------- teardown
@@ -594,6 +598,11 @@ cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream) {
   prm.K = a.K;
   prm.pair = a.nmat == 2 ? 0 : 1;
   prm.vec_store = (a.N % 8 == 0 && reinterpret_cast<uintptr_t>(a.y) % 16 == 0) ? 1 : 0;
+  prm.tma_store = (a.nmat == 1 && a.dst_row == nullptr && prm.vec_store) ? 1 : 0;
+  if (prm.tma_store) {
+    e = make_tmap_2d_bf16(&prm.tm_y, a.y, a.N, a.x_rows, kM, kEpiCols, /*swizzle128=*/false);
+    if (e != cudaSuccess) return e;
+  }
   prm.d_status = a.d_status;
   if (a.group == 32) return launch_ts_gs<32>(prm, stream);
   if (a.group == 64) return launch_ts_gs<64>(prm, stream);

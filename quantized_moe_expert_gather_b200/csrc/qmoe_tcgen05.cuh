@@ -132,6 +132,14 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// One dequantised A slice (16 or 32 columns) of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[16]) { tmem_st16(taddr, r); }
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st32(taddr, r); }
+
+// One epilogue piece of accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[32]) { tmem_ld32(taddr, v); }
+__device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
+
 // 8 packed 4-bit codes (one word, k ascending) -> 8 bf16 of q*s + b (one rounding each).
 __device__ __forceinline__ uint4 dequant_word4(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
   const uint32_t ws = w >> 4;
