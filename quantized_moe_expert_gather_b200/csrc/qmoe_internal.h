@@ -129,7 +129,10 @@ cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream); // tiles of 1
 bool qmm_tc_supported(const GemmArgs& a);
 // Tensor-core kernel with the dequantised weights as the MMA A operand in tensor memory,
 // for tiles of up to kTsTileRows rows: 4-bit codes, activations already in tile order.
-constexpr int kTsTileRows = 192;
+#ifndef QMOE_TS_TILE_ROWS
+#define QMOE_TS_TILE_ROWS 192
+#endif
+constexpr int kTsTileRows = QMOE_TS_TILE_ROWS;
 bool qmm_ts_supported(const GemmArgs& a);
 cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream);
 

@@ -56,8 +56,9 @@ constexpr int kNMax = kTsTileRows;               // routed rows per tile: MMA N 
 constexpr int kAtomK = 64;                       // k per 128-byte swizzle atom of bf16
 constexpr int kKC = QTS_KC;                      // k per step
 constexpr int kAtoms = kKC / kAtomK;             // activation atoms per step
-constexpr int kXBoxRows = 64;                    // activation rows per TMA box
-constexpr int kXBoxBytes = kXBoxRows * kAtomK * 2;  // 8 KB: 64 rows of one atom
+constexpr int kXBoxRows = 32;                    // activation box heights: multiples of 32 rows
+constexpr int kNXMaps = kNMax / kXBoxRows;       // one tensor map per box height
+constexpr int kXBoxBytes = kXBoxRows * kAtomK * 2;  // 4 KB: 32 rows of one atom
 constexpr int kXAtomBytes = kNMax * kAtomK * 2;     // 24 KB: one atom of a full tile
 constexpr int kXBytes = kAtoms * kXAtomBytes;       // per activation stage
 static_assert(kKC == 64 || kKC == 128, "step");
@@ -78,7 +79,10 @@ constexpr int kSbGroups = 8;                     // groups per scale/bias box
 constexpr int kSbBytes = 2 * 2 * 64 * kSbGroups * 2;  // [box][s|b][64 rows][8] bf16
 constexpr int kSbSlots = 2;
 constexpr int kACols = kKC / 2;                  // TMEM columns per A tile (bf16 pairs)
-constexpr int kASlots = 128 / kACols;            // dequantised A tiles in tensor memory
+#ifndef QTS_ASLOTS
+#define QTS_ASLOTS (128 / (QTS_KC / 2))
+#endif
+constexpr int kASlots = QTS_ASLOTS;              // dequantised A tiles in tensor memory
 constexpr int kTW = kKC / 16;                    // packed words per dequant thread and step
 constexpr int kDCol0 = kASlots * kACols;         // accumulators after the A tiles
 constexpr int kTmemCols = 512;
@@ -106,7 +110,7 @@ constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(k
 struct alignas(64) TsParams {
   CUtensorMap tm_w[2];      // packed codes [E*N, K/8] u32, box {32 words, 64 rows}, 128B swizzle
   CUtensorMap tm_sb[2][2];  // [stack][scales|biases] [E*N, K/group] bf16, box {8, 64}
-  CUtensorMap tm_x[3];      // activation rows [x_rows, K] bf16, box {64, 64*(i+1)}, 128B swizzle
+  CUtensorMap tm_x[kNXMaps];  // activation rows [x_rows, K] bf16, box {64, 32*(i+1)}, 128B swizzle
   CUtensorMap tm_y;         // output rows [x_rows, N] bf16, box {128, kEpiCols} (tma_store only)
   uint16_t* y;
   const uint32_t* dst_row;
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
     // ------------------------------------------------------- activation producer
     if (lane == 0) {
 #pragma unroll
-      for (int i = 0; i < 3; ++i) tma_prefetch_desc(&p.tm_x[i]);
+      for (int i = 0; i < kNXMaps; ++i) tma_prefetch_desc(&p.tm_x[i]);
       uint32_t it = 0;
       bool ab = false;
       int64_t cur = -1;
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
           if (*abort_flag) { ab = true; break; }
           const uint32_t s1 = it % kS1;
           if (!mbar_wait(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
-          // one box of 64, 128 or 192 rows: as many as the tile's MMA N reads
+          // per atom one box of as many 32-row blocks as the tile's MMA N reads
           mbar_arrive_expect_tx(&full1[s1], static_cast<uint32_t>(kAtoms * nbox * kXBoxBytes));
 #pragma unroll
           for (int a = 0; a < kAtoms; ++a)
@@ -573,7 +577,7 @@ cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream) {
   if (a.dense_rows <= 0 && a.bm != kNMax) return cudaErrorInvalidValue;  // tile table of kNMax rows
   TsParams prm{};
   cudaError_t e = cudaSuccess;
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < kNXMaps; ++i) {
     e = make_tmap_2d_bf16(&prm.tm_x[i], a.x, a.K, a.x_rows, kAtomK, kXBoxRows * (i + 1),
                           /*swizzle128=*/true);
     if (e != cudaSuccess) return e;
