@@ -49,6 +49,9 @@ QMM_CASES = [  # (M, N, K, bits, group)
     (3, 36, 1024, 4, 32), (1, 13, 96, 8, 32), (4, 24, 256, 8, 128), (40, 64, 256, 4, 64),
     (33, 50, 128, 8, 32), (64, 96, 4096, 4, 128), (16, 40, 64, 4, 64), (2, 1, 128, 8, 64),
     (17, 300, 640, 4, 64), (130, 256, 512, 4, 64), (300, 384, 1024, 8, 64),
+    # tensor-memory kernel edges: N not a multiple of 8 (element stores), several
+    # 192-row tiles with a ragged last one (TMA-stored full pieces), groups 32 and 128
+    (40, 37, 512, 4, 64), (200, 128, 1024, 4, 32), (400, 136, 2048, 4, 128),
 ]
 
 
