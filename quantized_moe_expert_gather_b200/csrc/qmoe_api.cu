@@ -466,6 +466,7 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   dn.dst_row = mode == 0 ? rb.order : nullptr;
   dn.tiles = rb.tiles;
   dn.num_tiles = rb.num_tiles;
+  dn.tiles_ready = true;  // written by the routing kernel, before the up/gate launch
   dn.d_status = d_status;
   // With distinct experts per token one expert receives at most T rows.  The bound only
   // picks the plan: any routing is served correctly by either kernel.

@@ -118,6 +118,10 @@ struct GemmArgs {
   int64_t dense_rows = 0;            // > 0: no tile table, rows [0, dense_rows), expert 0
   int64_t max_tiles = 0;             // host upper bound of the tile count
   int bm = 8;                        // rows per tile the table was built with
+  // The tile table was written before the kernel launched just before this one (the
+  // down projection after the up/gate launch): with the weights, it may be read before
+  // that kernel completes.
+  bool tiles_ready = false;
   int* d_status = nullptr;
 };
 cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream);   // tiles of <= 16 rows

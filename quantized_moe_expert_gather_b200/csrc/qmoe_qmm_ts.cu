@@ -122,6 +122,7 @@ struct alignas(64) TsParams {
   int vec_store;            // y rows start 16-byte aligned: 8 channels per store
   int tma_store;            // one stack, rows in tile order (no dst_row), vec_store: full
                             // epilogue pieces leave by TMA tensor stores
+  int early_weights;        // tile table older than the previous kernel (or none)
   int* d_status;
   ProfSlot* prof;
 };
@@ -207,8 +208,12 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_sh;
-  // inputs (tile table, activations) may come from the kernel before this one
-  griddep_wait();
+  // Inputs (tile table, activations) may come from the kernel before this one.  When the
+  // tile table is older (or there is none), the weight producer and the dequant warps --
+  // which read only the table and the weights, never written by the kernel just before --
+  // start at once, overlapping the tail of that kernel.
+  if (!(p.early_weights && (warp == kProdWWarp || (warp >= kDqWarp0 && warp < kDqWarp0 + kDqWarps))))
+    griddep_wait();
   griddep_launch_dependents();
   if (threadIdx.x == 0) prof_start(p.prof);
 
@@ -601,6 +606,7 @@ cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream) {
   prm.N = a.N;
   prm.K = a.K;
   prm.pair = a.nmat == 2 ? 0 : 1;
+  prm.early_weights = (a.dense_rows > 0 || a.tiles_ready) ? 1 : 0;
   prm.vec_store = (a.N % 8 == 0 && reinterpret_cast<uintptr_t>(a.y) % 16 == 0) ? 1 : 0;
   prm.tma_store = (a.nmat == 1 && a.dst_row == nullptr && prm.vec_store) ? 1 : 0;
   if (prm.tma_store) {

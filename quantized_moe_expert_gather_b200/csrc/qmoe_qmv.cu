@@ -111,6 +111,7 @@ struct alignas(64) QmvParams {
   int code3d;                   // codes by one 3-D box per 16-row block (else one 2-D box per 128 B)
   int sb_tma;                   // scales/biases by TMA (row pitch a multiple of 16 bytes)
   int sb_vec;                   // else: byte width of the copy pieces (2: plain copies)
+  int early_weights;            // the producer may stream before the previous kernel ends
   int* d_status;
   ProfSlot* prof;
 };
@@ -176,11 +177,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  // Inputs (tile table, activations) may come from the kernel before this one.  A dense
-  // launch has no tile table, and its weights are never written by the kernel launched
-  // just before it: there the producer streams weights at once, overlapping the tail of
-  // that kernel, and only the roles that read activations or write y wait.
-  if (!(p.dense_rows > 0 && warp == kConsumerWarps)) griddep_wait();
+  // Inputs (tile table, activations) may come from the kernel before this one.  When the
+  // tile table is older (a dense launch has none; the down projection's was written
+  // before the up/gate launch) and the weights are never written by the kernel launched
+  // just before it, the producer streams weights at once, overlapping the tail of that
+  // kernel, and only the roles that read activations or write y wait.
+  if (!(p.early_weights && warp == kConsumerWarps)) griddep_wait();
   griddep_launch_dependents();
   if (threadIdx.x == 0) prof_start(p.prof);
 
@@ -694,6 +696,7 @@ cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
   prm.tiles = a.tiles;
   prm.num_tiles = a.num_tiles;
   prm.dense_rows = a.dense_rows;
+  prm.early_weights = (a.dense_rows > 0 || a.tiles_ready) ? 1 : 0;
   prm.N = a.N;
   prm.K = a.K;
   prm.E = a.E;
