@@ -83,10 +83,16 @@ constexpr int kACols = kKC / 2;                  // TMEM columns per A tile (bf1
 #define QTS_ASLOTS (128 / (QTS_KC / 2))
 #endif
 constexpr int kASlots = QTS_ASLOTS;              // dequantised A tiles in tensor memory
-constexpr int kTW = kKC / 16;                    // packed words per dequant thread and step
+#ifndef QTS_DQ_WARPS
+#define QTS_DQ_WARPS 8
+#endif
+constexpr int kDqWarps = QTS_DQ_WARPS;           // 8 or 16
+constexpr int kDqParts = kDqWarps / 4;           // k slices of a step, one per warp of a quarter
+constexpr int kTW = kKC / 8 / kDqParts;          // packed words per dequant thread and step
+static_assert((kDqWarps == 8 || kDqWarps == 16) && kTW % 4 == 0, "dequant split");
 constexpr int kDCol0 = kASlots * kACols;         // accumulators after the A tiles
 constexpr int kTmemCols = 512;
-constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps = 8;
+constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6;
 constexpr int kProdWWarp = kDqWarp0 + kDqWarps;       // 14: packed codes, scales, biases
 constexpr int kEpi2Warp0 = kProdWWarp + 1;            // 15-18: second epilogue group
 constexpr int kThreads = (kEpi2Warp0 + kEpiWarps) * 32;  // 608
@@ -155,7 +161,7 @@ template <int GS>
 __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_constant__ TsParams p) {
   constexpr int KS_SB = kSbGroups * GS / kKC;  // steps per scale/bias window
   static_assert((kSbGroups * GS) % kKC == 0 && KS_SB >= 1, "group size");
-  constexpr int GPT = (kKC / 2) >= GS ? (kKC / 2) / GS : 1;  // groups of a thread's k per step
+  constexpr int GPT = (kTW * 8) >= GS ? (kTW * 8) / GS : 1;  // groups of a thread's k per step
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -393,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
         // piece c at c ^ (rr & 7)
         const uint8_t* rowp = smem + kOffP + sp * kPBytes + m * 64 * 128 + rr * 128;
         // the thread's k lie in GPT groups, the first at g0 of the scale window
-        const int g0 = (static_cast<int>((ks * kKC) % (kSbGroups * GS)) + part * (kKC / 2)) / GS;
+        const int g0 = (static_cast<int>((ks * kKC) % (kSbGroups * GS)) + part * (kTW * 8)) / GS;
         const uint16_t* sbw = reinterpret_cast<const uint16_t*>(smem + kOffSb + e * kSbBytes);
         __nv_bfloat162 s2[GPT], b2[GPT];
         load_group_pairs<GPT>(sbw + (m * 2 * 64 + rr) * kSbGroups + g0, s2);
