@@ -29,7 +29,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "bf16_from_f32", "f32_from_bf16", "pack_codes", "unpack_codes", "quantize",
+    "CODE_BITS", "bf16_from_f32", "f32_from_bf16", "pack_codes", "unpack_codes", "quantize",
     "dequantize", "qmm", "gather_qmm", "gather_mm", "sort_by_expert", "tile_table",
     "silu", "switch_glu", "moe_combine", "moe_combine_stock", "sigmoid",
 ]
@@ -58,33 +58,41 @@ def bf16_from_f32(f: np.ndarray) -> np.ndarray:
 
 # -------------------------------------------------------------------------- packing
 
+# Bit widths of [P3] (``const BITS``); 7 is rejected there (``quantize(64, 7)`` fails).
+CODE_BITS = (1, 2, 3, 4, 5, 6, 8)
+
+
 def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
     """Pack integer codes along the last axis into uint32 words.
 
-    Code j of a word occupies bits [(j mod 32/bits)*bits, ...): the first code of a
-    word sits in its least significant bits.  The packed shape is
-    ``[..., cols*bits/32]`` as in [P3] ``round_trip_error_is_about_half_a_step``.
+    The codes of a row form one least-significant-bit-first bit stream: code j
+    occupies stream bits [j*bits, (j+1)*bits), and stream bit i is bit (i mod 32) of
+    word i // 32.  For widths that divide 32 this is "code j of a word in bits
+    [(j mod 32/bits)*bits, ...)"; for 3, 5 and 6 bits a code may straddle two words.
+    The packed shape is ``[..., cols*bits/32]`` for every width, as [P3]
+    ``round_trip_error_is_about_half_a_step`` asserts.
     """
-    assert bits in (4, 8)
-    per = 32 // bits
-    codes = np.asarray(codes, dtype=np.uint64)
-    assert codes.shape[-1] % per == 0
-    assert codes.max(initial=0) < (1 << bits)
-    grouped = codes.reshape(codes.shape[:-1] + (codes.shape[-1] // per, per))
-    words = np.zeros(grouped.shape[:-1], dtype=np.uint64)
-    for j in range(per):
-        words |= grouped[..., j] << np.uint64(j * bits)
-    return words.astype(np.uint32)
+    assert bits in CODE_BITS
+    codes = np.asarray(codes, dtype=np.int64)
+    assert (codes.shape[-1] * bits) % 32 == 0
+    assert codes.min(initial=0) >= 0 and codes.max(initial=0) < (1 << bits)
+    # stream[..., j*bits + i] = bit i of code j
+    shifts = np.arange(bits, dtype=np.int64)
+    stream = ((codes[..., :, None] >> shifts) & 1).reshape(codes.shape[:-1] + (-1,))
+    stream = stream.reshape(stream.shape[:-1] + (stream.shape[-1] // 32, 32)).astype(np.uint64)
+    weights = np.left_shift(np.uint64(1), np.arange(32, dtype=np.uint64))
+    return (stream * weights).sum(axis=-1).astype(np.uint32)
 
 
 def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
     """Inverse of :func:`pack_codes`; returns int64 codes."""
-    per = 32 // bits
+    assert bits in CODE_BITS
     w = np.asarray(words, dtype=np.uint64)
-    mask = np.uint64((1 << bits) - 1)
-    parts = [(w >> np.uint64(j * bits)) & mask for j in range(per)]
-    out = np.stack(parts, axis=-1)
-    return out.reshape(w.shape[:-1] + (w.shape[-1] * per,)).astype(np.int64)
+    stream = (w[..., :, None] >> np.arange(32, dtype=np.uint64)) & np.uint64(1)
+    stream = stream.reshape(w.shape[:-1] + (-1,))
+    per_code = stream.reshape(stream.shape[:-1] + (stream.shape[-1] // bits, bits))
+    weights = np.left_shift(np.uint64(1), np.arange(bits, dtype=np.uint64))
+    return (per_code * weights).sum(axis=-1).astype(np.int64)
 
 
 # ---------------------------------------------------------------------- quantisation
@@ -117,7 +125,7 @@ def quantize(w: np.ndarray, group: int, bits: int, scale_dtype: str = "bf16"):
     step 2, half-even rint, codes from stored values): they are the plainest
     reading that meets every invariant the pages state.
     """
-    assert bits in (4, 8) and group in (32, 64, 128)
+    assert bits in CODE_BITS and group in (32, 64, 128)
     w = np.asarray(w, dtype=np.float32)
     assert w.ndim == 2 and w.shape[1] % group == 0
     rows, cols = w.shape

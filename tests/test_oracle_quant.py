@@ -32,9 +32,42 @@ def test_pack_layout_hand_words():
     assert O.pack_codes(np.array([[1, 2, 3, 4]]), 8)[0, 0] == 0x04030201
     assert O.pack_codes(np.array([[15, 0, 0, 0, 0, 0, 0, 1]]), 4)[0, 0] == 0x1000000F
     rng = np.random.default_rng(3)
-    for bits in (4, 8):
+    for bits in O.CODE_BITS:
         c = rng.integers(0, 1 << bits, size=(3, 64))
         assert np.array_equal(O.unpack_codes(O.pack_codes(c, bits), bits), c)
+
+
+def _one_code(n, j, v):
+    c = np.zeros((1, n), np.int64)
+    c[0, j] = v
+    return c
+
+
+def test_pack_bit_stream_hand_words():
+    """Codes form one least-significant-bit-first stream per row (code j at stream bits
+    [j*bits, (j+1)*bits)); [P3] fixes the packed row at cols*bits/32 words for every
+    width, so 3-, 5- and 6-bit codes straddle words.  Words worked out by hand."""
+    # 1 bit: codes 0 and 31 set
+    c = np.zeros((1, 32), np.int64)
+    c[0, 0] = c[0, 31] = 1
+    assert [int(v) for v in O.pack_codes(c, 1)[0]] == [0x80000001]
+    # 2 bits: 0,1,2,3 repeated -> byte 0b11100100
+    assert [int(v) for v in O.pack_codes(np.arange(16)[None] % 4, 2)[0]] == [0xE4E4E4E4]
+    # 3 bits: code 10 = 0b111 sits at stream bits 30..32
+    assert [int(v) for v in O.pack_codes(_one_code(32, 10, 7), 3)[0]] == [0xC0000000, 0x1, 0]
+    # 5 bits: code 6 = 0b10101 at stream bits 30..34
+    assert [int(v) for v in O.pack_codes(_one_code(32, 6, 21), 5)[0]] == [0x40000000, 0x5, 0, 0, 0]
+    # 6 bits: code 5 = 0b110011 at stream bits 30..35
+    assert [int(v) for v in O.pack_codes(_one_code(32, 5, 51), 6)[0]] == \
+        [0xC0000000, 0xC, 0, 0, 0, 0]
+    for bits in (3, 5, 6):
+        assert O.pack_codes(np.zeros((2, 64), np.int64), bits).shape == (2, 2 * bits)
+
+
+def test_seven_bits_is_rejected():
+    """[P3] rejected_arguments: quantize(64, 7) fails."""
+    with pytest.raises(AssertionError):
+        O.quantize(np.zeros((1, 64), np.float32), 64, 7)
 
 
 def test_quantize_hand_example():
@@ -46,7 +79,7 @@ def test_quantize_hand_example():
     assert np.array_equal(O.dequantize(packed, s, b, 32, 4), w)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", O.CODE_BITS)
 @pytest.mark.parametrize("group", [32, 64, 128])
 @pytest.mark.parametrize("dist", ["uniform", "normal"])
 def test_round_trip_error_is_about_half_a_step(bits, group, dist):
@@ -66,24 +99,26 @@ def test_round_trip_error_is_about_half_a_step(bits, group, dist):
     assert err.sum() <= step.sum() / 2
 
 
-def test_quantize_constant_negative_and_zero_spanning_groups():
+@pytest.mark.parametrize("bits", O.CODE_BITS)
+def test_quantize_constant_negative_and_zero_spanning_groups(bits):
     """nuvec-core quantized.rs quantize_snaps_zero_and_handles_constant_and_one_signed_groups."""
     v = [0.75] * 32 + [-1.0 - i / 8 for i in range(32)] + [i / 31 - 0.25 for i in range(32)]
     w = np.array(v, np.float32).reshape(3, 32)
-    packed, s, b = O.quantize(w, 32, 4, scale_dtype="f32")
-    back = O.dequantize(packed, s, b, 32, 4)
+    packed, s, b = O.quantize(w, 32, bits, scale_dtype="f32")
+    back = O.dequantize(packed, s, b, 32, bits)
     assert np.all(np.abs(back[0] - 0.75) < 1e-6)
     # all-negative group stays within one step
     assert np.all(np.abs(back[1] - w[1]) <= abs(s[1, 0]) * 1.0001)
-    # zero is representable in a group that spans it
-    codes = O.unpack_codes(packed, 4)[2].astype(np.float64)
-    assert np.any(np.abs(codes * s[2, 0] + b[2, 0]) < 1e-7)
+    # zero is exactly representable in a group that spans it: some code in [0, 2^bits)
+    # restores it to within 1e-7
+    q = np.arange(1 << bits, dtype=np.float64)
+    assert np.min(np.abs(q * s[2, 0] + b[2, 0])) < 1e-7
 
 
 def test_quantize_codes_in_range_and_bf16_storage_close_to_f32():
     rng = np.random.default_rng(7)
     w = rng.standard_normal((16, 256)).astype(np.float32)
-    for bits in (4, 8):
+    for bits in O.CODE_BITS:
         p32, s32, b32 = O.quantize(w, 64, bits, "f32")
         p16, s16, b16 = O.quantize(w, 64, bits, "bf16")
         c = O.unpack_codes(p16, bits)
@@ -98,7 +133,7 @@ def test_quantize_codes_in_range_and_bf16_storage_close_to_f32():
 def test_dequantize_dyadic_closed_form():
     """q*s + b with dyadic s and b is exact: compare with integer arithmetic."""
     rng = np.random.default_rng(11)
-    for bits in (4, 8):
+    for bits in O.CODE_BITS:
         codes = rng.integers(0, 1 << bits, size=(5, 128))
         packed = O.pack_codes(codes, bits)
         sq = rng.integers(1, 64, size=(5, 2))          # s = sq / 256
