@@ -24,10 +24,14 @@
  *   - Errors found on the device never trap: they are OR-ed into the optional
  *     `int* d_status` (device memory, caller-zeroed) as QMOE_DEV_* bits, and the
  *     rows concerned are written as zeros.
- *   - Supported codecs: bits in {4, 8}; group in {32, 64, 128}; K a positive
- *     multiple of the group size (QMOE_ERR_UNSUPPORTED / QMOE_ERR_ARG otherwise).
- *     Packed layout: code j of a uint32 word occupies bits
- *     [(j mod 32/bits)*bits, ...), so W [rows, K] packs to [rows, K*bits/32].
+ *   - Supported codecs: group in {32, 64, 128}; bits in {1, 2, 3, 4, 5, 6, 8} for
+ *     qmoe_quantize / qmoe_dequantize (the widths of nuvec-core's quantisation tests),
+ *     {4, 8} for the matmul calls (others return QMOE_ERR_UNSUPPORTED); K a positive
+ *     multiple of the group.  Packed layout: the codes of a row form one
+ *     least-significant-bit-first bit stream, code j at stream bits [j*bits, (j+1)*bits)
+ *     and stream bit i in bit (i mod 32) of word i/32 -- for 4 and 8 bits, code j of a
+ *     word in bits [(j mod 32/bits)*bits, ...); 3-, 5- and 6-bit codes may straddle two
+ *     words -- so W [rows, K] packs to [rows, K*bits/32].
  */
 #ifndef QMOE_H_
 #define QMOE_H_

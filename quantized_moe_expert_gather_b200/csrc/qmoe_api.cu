@@ -10,13 +10,17 @@ using namespace qmoe;
 
 namespace {
 
+bool group_ok(int group) { return group == 32 || group == 64 || group == 128; }
+// quantize / dequantize: every width of the quantisation tests (7 is rejected there)
 bool codec_ok(int group, int bits) {
-  return (bits == 4 || bits == 8) && (group == 32 || group == 64 || group == 128);
+  return (bits >= 1 && bits <= 8 && bits != 7) && group_ok(group);
 }
+// the matmul kernels: 4- and 8-bit codes
+bool matmul_codec_ok(int group, int bits) { return (bits == 4 || bits == 8) && group_ok(group); }
 
 // K must be a positive multiple of the group size.
 int check_codec(int64_t K, int group, int bits) {
-  if (!codec_ok(group, bits)) return QMOE_ERR_UNSUPPORTED;
+  if (!matmul_codec_ok(group, bits)) return QMOE_ERR_UNSUPPORTED;
   if (K <= 0 || K % group != 0) return QMOE_ERR_ARG;
   return QMOE_OK;
 }

@@ -78,17 +78,23 @@ __global__ void quantize_kernel(const T* __restrict__ w, int64_t rows, int64_t c
   const float b_st = round_to_storage<T>(bias);
   store_val(scales, gid, scale);
   store_val(biases, gid, bias);
-  constexpr int PER = 32 / BITS;
-  uint32_t* dst = codes + (row * cols + g * group) / PER;
-  for (int wi = 0; wi < group / PER; ++wi) {
-    uint32_t word = 0;
-    for (int j = 0; j < PER; ++j) {
-      const float v = load_val(src, wi * PER + j);
-      float q = rintf(__fdiv_rn(__fsub_rn(v, b_st), s_st));
-      q = fminf(fmaxf(q, 0.0f), n);
-      word |= static_cast<uint32_t>(q) << (j * BITS);
+  // The row's codes are one least-significant-bit-first bit stream (code j at stream
+  // bits [j*BITS, (j+1)*BITS)); a group of a multiple of 32 codes fills whole words, so
+  // each thread writes its own words.
+  uint32_t* dst = codes + (row * cols + g * group) * BITS / 32;
+  uint64_t acc = 0;
+  int nacc = 0;
+  for (int i = 0; i < group; ++i) {
+    const float v = load_val(src, i);
+    float q = rintf(__fdiv_rn(__fsub_rn(v, b_st), s_st));
+    q = fminf(fmaxf(q, 0.0f), n);
+    acc |= static_cast<uint64_t>(q) << nacc;
+    nacc += BITS;
+    if (nacc >= 32) {
+      *dst++ = static_cast<uint32_t>(acc);
+      acc >>= 32;
+      nacc -= 32;
     }
-    dst[wi] = word;
   }
 }
 
@@ -112,6 +118,43 @@ __global__ void dequantize_kernel(const uint32_t* __restrict__ codes, const S* _
   }
 }
 
+// Any width: one thread per element, reading the (up to two) words its code spans.
+template <typename S, typename O>
+__global__ void dequantize_stream_kernel(const uint32_t* __restrict__ codes,
+                                         const S* __restrict__ scales,
+                                         const S* __restrict__ biases, int64_t rows, int64_t cols,
+                                         int group, int bits, O* __restrict__ out) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= rows * cols) return;
+  const int64_t row = idx / cols, j = idx % cols;
+  const uint32_t* rw = codes + row * (cols * bits / 32);
+  const int64_t bit = j * bits;
+  const int64_t w = bit >> 5;
+  const int o = static_cast<int>(bit & 31);
+  uint64_t v = rw[w];
+  if (o + bits > 32) v |= static_cast<uint64_t>(rw[w + 1]) << 32;
+  const float q = static_cast<float>((v >> o) & ((1ull << bits) - 1));
+  const int64_t gidx = row * (cols / group) + j / group;
+  store_val(out, idx, __fadd_rn(__fmul_rn(q, load_val(scales, gidx)), load_val(biases, gidx)));
+}
+
+template <typename T>
+cudaError_t launch_quantize_t(const T* wp, int64_t rows, int64_t cols, int group, int bits,
+                              uint32_t* codes, T* sp, T* bp, unsigned blocks, int threads,
+                              cudaStream_t stream) {
+  switch (bits) {
+    case 1: quantize_kernel<T, 1><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp); break;
+    case 2: quantize_kernel<T, 2><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp); break;
+    case 3: quantize_kernel<T, 3><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp); break;
+    case 4: quantize_kernel<T, 4><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp); break;
+    case 5: quantize_kernel<T, 5><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp); break;
+    case 6: quantize_kernel<T, 6><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp); break;
+    case 8: quantize_kernel<T, 8><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const void* w, bool w_f32, int64_t rows, int64_t cols, int group,
@@ -121,23 +164,14 @@ cudaError_t launch_quantize(const void* w, bool w_f32, int64_t rows, int64_t col
   if (n == 0) return cudaSuccess;
   const int threads = 128;
   const unsigned blocks = static_cast<unsigned>((n + threads - 1) / threads);
-  if (w_f32) {
-    auto* wp = static_cast<const float*>(w);
-    auto* sp = static_cast<float*>(scales);
-    auto* bp = static_cast<float*>(biases);
-    if (bits == 4)
-      quantize_kernel<float, 4><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp);
-    else
-      quantize_kernel<float, 8><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp);
-  } else {
-    auto* wp = static_cast<const uint16_t*>(w);
-    auto* sp = static_cast<uint16_t*>(scales);
-    auto* bp = static_cast<uint16_t*>(biases);
-    if (bits == 4)
-      quantize_kernel<uint16_t, 4><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp);
-    else
-      quantize_kernel<uint16_t, 8><<<blocks, threads, 0, stream>>>(wp, rows, cols, group, codes, sp, bp);
-  }
+  const cudaError_t e =
+      w_f32 ? launch_quantize_t(static_cast<const float*>(w), rows, cols, group, bits, codes,
+                                static_cast<float*>(scales), static_cast<float*>(biases), blocks,
+                                threads, stream)
+            : launch_quantize_t(static_cast<const uint16_t*>(w), rows, cols, group, bits, codes,
+                                static_cast<uint16_t*>(scales), static_cast<uint16_t*>(biases),
+                                blocks, threads, stream);
+  if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }
@@ -146,8 +180,16 @@ namespace {
 template <typename S, typename O>
 void dequant_dispatch(const uint32_t* codes, const void* s, const void* b, int64_t rows,
                       int64_t cols, int group, int bits, void* out, cudaStream_t stream) {
-  const int64_t n = rows * (cols * bits / 32);
   const int threads = 256;
+  if (bits != 4 && bits != 8) {
+    const int64_t ne = rows * cols;
+    dequantize_stream_kernel<S, O><<<static_cast<unsigned>((ne + threads - 1) / threads), threads,
+                                     0, stream>>>(codes, static_cast<const S*>(s),
+                                                  static_cast<const S*>(b), rows, cols, group,
+                                                  bits, static_cast<O*>(out));
+    return;
+  }
+  const int64_t n = rows * (cols * bits / 32);
   const unsigned blocks = static_cast<unsigned>((n + threads - 1) / threads);
   if (bits == 4)
     dequantize_kernel<S, O, 4><<<blocks, threads, 0, stream>>>(

@@ -25,7 +25,7 @@ def _weights(rng, rows, cols, group):
     return w
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", O.CODE_BITS)
 @pytest.mark.parametrize("group", [32, 64, 128])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_quantize_dequantize_bit_exact(gpu_lib, bits, group, dtype):
@@ -53,6 +53,20 @@ def test_quantize_dequantize_bit_exact(gpu_lib, bits, group, dtype):
     assert np.array_equal(d32.cpu().numpy().view(np.uint32), want_d.view(np.uint32))
     d16 = q.qmoe_dequantize(codes, s, b, group, bits, out_dtype=torch.bfloat16)
     assert np.array_equal(host_bits16(d16), O.bf16_from_f32(want_d))
+
+
+def test_codec_widths_outside_the_kernels_are_rejected(gpu_lib):
+    """7 bits is rejected by the codec ([P3] rejected_arguments); widths other than 4
+    and 8 quantise and dequantise but are rejected by the matmul calls."""
+    q = gpu_lib
+    w = torch.zeros((2, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+        q.qmoe_quantize(w, 64, 7)
+    codes, s, b = q.qmoe_quantize(w.to(torch.bfloat16), 64, 3)
+    assert codes.shape == (2, 6)
+    x = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+        q.qmoe_qmm(x, codes, s, b, 64, 3)
 
 
 @pytest.mark.parametrize("R,E", [(1, 1), (37, 5), (1024, 288), (1025, 256), (4099, 8),
