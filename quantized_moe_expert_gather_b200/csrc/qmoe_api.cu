@@ -15,8 +15,11 @@ bool group_ok(int group) { return group == 32 || group == 64 || group == 128; }
 bool codec_ok(int group, int bits) {
   return (bits >= 1 && bits <= 8 && bits != 7) && group_ok(group);
 }
-// the matmul kernels: 4- and 8-bit codes
-bool matmul_codec_ok(int group, int bits) { return (bits == 4 || bits == 8) && group_ok(group); }
+// the matmul kernels: 4- and 8-bit codes, and 2-bit codes in groups of 64 or 128
+bool matmul_codec_ok(int group, int bits) {
+  if (bits == 2) return group == 64 || group == 128;
+  return (bits == 4 || bits == 8) && group_ok(group);
+}
 
 // K must be a positive multiple of the group size.
 int check_codec(int64_t K, int group, int bits) {

@@ -71,13 +71,20 @@ struct Cfg {
   static constexpr int THREADS = (CW + 2) * 32;  // consumers, producer, epilogue
   static constexpr int KB_BYTES = GS * BITS / 8;                 // one group of one row
   // 1 KB of each row per stage (512 B with two token sets, whose doubled register
-  // arrays would otherwise spill), at least one group per consumer warp
-  static constexpr int CHUNK_ROW_BYTES = std::max(NT == 2 ? 512 : 1024, KB_BYTES * CW);
+  // arrays would otherwise spill; half that for 2-bit codes, whose activations per
+  // code byte are twice as many), at least one group per consumer warp
+  static constexpr int CHUNK_ROW_BYTES =
+      std::max((NT == 2 ? 512 : 1024) / (BITS == 2 ? 2 : 1), KB_BYTES * CW);
   static constexpr int KB_PER_CHUNK = CHUNK_ROW_BYTES / KB_BYTES;
   static constexpr int KB_PER_WARP = KB_PER_CHUNK / CW;
   static constexpr int BOXES = CHUNK_ROW_BYTES / 128;
   static constexpr int LANE_BYTES = KB_BYTES / 4;                // per row, per lane
   static constexpr int WORDS = LANE_BYTES / 4;
+  // activation vectors (16 B of bf16 for 2- and 4-bit codes, 8 B for 8-bit) per code word
+  static constexpr int XW = BITS == 2 ? 2 : 1;
+  // MMA k-steps per code word: 16 codes (2-bit) -> 4, 8 codes (4-bit) -> 2, 4 codes (8-bit)
+  // -> 2 (low and high nibbles of the same activation pairs)
+  static constexpr int MPW = BITS == 2 ? 4 : 2;
   static constexpr int CODE_BYTES = NMAT * BOXES * 2048;
   static constexpr int SB_BYTES = NMAT * 2 * kRows * KB_PER_CHUNK * 2;
   static constexpr int STAGE_BYTES = ((CODE_BYTES + SB_BYTES) + 1023) / 1024 * 1024;
@@ -89,7 +96,9 @@ struct Cfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RED_BYTES + 2 * STAGES * 8 + 4 * 8 + 64;
   static constexpr uint32_t TMA_BYTES = CODE_BYTES;
   static_assert((kRows * KB_PER_CHUNK * 2) % 128 == 0, "scale/bias TMA boxes must stay 128-byte aligned");
-  static constexpr float OFFSET = BITS == 4 ? 128.0f : 2176.0f;
+  static constexpr float OFFSET = BITS == 8 ? 2176.0f : 128.0f;
+  static_assert(BITS == 2 || BITS == 4 || BITS == 8, "code width");
+  static_assert(LANE_BYTES >= 4, "a lane's share of a group must be whole words");
   static_assert(STAGES >= 3, "too few pipeline stages");
   static_assert(KB_PER_WARP >= 1, "chunk smaller than one group per warp");
 };
@@ -354,8 +363,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
   // Activation values of one chunk for this lane: [k-block][token set][word]; 16 B per
   // 4-bit word (8 codes), 8 B per 8-bit word (4 codes).  Two buffers alternate: one is
   // consumed while the loads of the next chunk land in the other.
-  using XV = typename std::conditional<BITS == 4, uint4, uint2>::type;
-  using XBuf = XV[C::KB_PER_WARP][NT][C::WORDS];
+  using XV = typename std::conditional<BITS == 8, uint2, uint4>::type;
+  using XBuf = XV[C::KB_PER_WARP][NT][C::WORDS * C::XW];
   XBuf xa, xb;
 
   // Shared-memory offsets of this lane, fixed for the kernel.  The warp's group i sits
@@ -401,8 +410,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int j = 0; j < C::WORDS; ++j) {
-          if constexpr (BITS == 4) {
+        for (int j = 0; j < C::WORDS * C::XW; ++j) {
+          if constexpr (BITS != 8) {  // 8 activations per vector, XW vectors per code word
             dst[i][nt][j] = make_uint4(0, 0, 0, 0);
             if (rows[nt] != nullptr && live)
               dst[i][nt][j] = ldg_nc_v4(rows[nt] + ch * CHUNK_ELEMS + i * C::CW * GS + 8 * j);
@@ -485,12 +494,22 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
       for (int i = 0; i < C::KB_PER_WARP; ++i) {
         if (warp + C::CW * i >= nkb) break;
         // ---- B operand: x values of this lane's codes, permuted to the MMA k order
-        uint32_t bfr[NT][C::WORDS][2][2];
+        uint32_t bfr[NT][C::WORDS][C::MPW][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
           for (int j = 0; j < C::WORDS; ++j) {
-            if constexpr (BITS == 4) {
+            if constexpr (BITS == 2) {
+              // 16 activations of a 16-code word: MMA m pairs codes (2m, 2m+8) and
+              // (2m+1, 2m+9), the halves of component m of the two vectors
+              const uint4 v0 = xc[i][nt][2 * j], v1 = xc[i][nt][2 * j + 1];
+              const uint32_t c0[4] = {v0.x, v0.y, v0.z, v0.w}, c1[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+              for (int mm = 0; mm < 4; ++mm) {
+                bfr[nt][j][mm][0] = prmt(c0[mm], c1[mm], 0x5410);
+                bfr[nt][j][mm][1] = prmt(c0[mm], c1[mm], 0x7632);
+              }
+            } else if constexpr (BITS == 4) {
               const uint4 v = xc[i][nt][j];
               bfr[nt][j][0][0] = prmt(v.x, v.z, 0x5410);
               bfr[nt][j][0][1] = prmt(v.x, v.z, 0x7632);
@@ -514,8 +533,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
           const uint32_t ones[4] = {ONES, ONES, ONES, ONES};
 #pragma unroll
           for (int j = 0; j < C::WORDS; ++j) {
-            mma_bf16_16816(cx[nt], ones, bfr[nt][j][0][0], bfr[nt][j][0][1]);
-            if constexpr (BITS == 4) mma_bf16_16816(cx[nt], ones, bfr[nt][j][1][0], bfr[nt][j][1][1]);
+            // 8-bit codes reuse one activation pair for both nibbles: count it once
+#pragma unroll
+            for (int mm = 0; mm < (BITS == 8 ? 1 : C::MPW); ++mm)
+              mma_bf16_16816(cx[nt], ones, bfr[nt][j][mm][0], bfr[nt][j][mm][1]);
           }
         }
 #pragma unroll
@@ -545,8 +566,18 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
             for (int i2 = 0; i2 < 4; ++i2) cacc[nt][i2] = 0.f;
 #pragma unroll
           for (int j = 0; j < C::WORDS; ++j) {
-            uint32_t a[2][4];
-            if constexpr (BITS == 4) {
+            uint32_t a[C::MPW][4];
+            if constexpr (BITS == 2) {
+              // pair i = (code i, code i+8) from the word shifted by 2i, as bf16 128 + q
+              const uint32_t M2 = 0x00030003u, MAG = 0x43004300u;
+#pragma unroll
+              for (int mm = 0; mm < 4; ++mm) {
+                a[mm][0] = and_or(wg[j] >> (4 * mm), M2, MAG);
+                a[mm][1] = and_or(wg8[j] >> (4 * mm), M2, MAG);
+                a[mm][2] = and_or(wg[j] >> (4 * mm + 2), M2, MAG);
+                a[mm][3] = and_or(wg8[j] >> (4 * mm + 2), M2, MAG);
+              }
+            } else if constexpr (BITS == 4) {
               const uint32_t M4 = 0x000F000Fu, MAG = 0x43004300u;
               a[0][0] = and_or(wg[j], M4, MAG);
               a[0][1] = and_or(wg8[j], M4, MAG);
@@ -568,10 +599,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
               a[1][3] = and_or(wg8[j] >> 12, M4, HI);
             }
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              mma_bf16_16816(cacc[nt], a[0], bfr[nt][j][0][0], bfr[nt][j][0][1]);
-              mma_bf16_16816(cacc[nt], a[1], bfr[nt][j][1][0], bfr[nt][j][1][1]);
-            }
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int mm = 0; mm < C::MPW; ++mm)
+                mma_bf16_16816(cacc[nt], a[mm], bfr[nt][j][mm][0], bfr[nt][j][mm][1]);
           }
           // scales and biases of rows g and g+8 for this group
           const uint16_t* sm = sb + (m * 2) * kRows * C::KB_PER_CHUNK + C::CW * i;
@@ -704,6 +735,10 @@ cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
   prm.sb_vec = (gpr % 8 == 0) ? 16 : (gpr % 4 == 0) ? 8 : (gpr % 2 == 0) ? 4 : 2;
   prm.d_status = a.d_status;
   const int nt = a.bm > 8 ? 2 : 1;
+  if (a.bits == 2) {  // groups of 64 or 128 (a lane's share of a group is whole words)
+    if (a.group == 64) return launch_bits_gs<2, 64>(prm, a, nt, stream);
+    return launch_bits_gs<2, 128>(prm, a, nt, stream);
+  }
   if (a.bits == 4) {
     if (a.group == 32) return launch_bits_gs<4, 32>(prm, a, nt, stream);
     if (a.group == 64) return launch_bits_gs<4, 64>(prm, a, nt, stream);

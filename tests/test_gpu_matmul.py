@@ -52,6 +52,8 @@ QMM_CASES = [  # (M, N, K, bits, group)
     # tensor-memory kernel edges: N not a multiple of 8 (element stores), several
     # 192-row tiles with a ragged last one (TMA-stored full pieces), groups 32 and 128
     (40, 37, 512, 4, 64), (200, 128, 1024, 4, 32), (400, 136, 2048, 4, 128),
+    # 2-bit codes (streaming kernel, one and two token sets, groups 64 and 128)
+    (1, 64, 512, 2, 64), (5, 96, 1024, 2, 128), (12, 64, 512, 2, 64), (40, 37, 1024, 2, 128),
 ]
 
 
@@ -132,6 +134,7 @@ GATHER_CASES = [  # (E, N, K, M, batches, sorted, bits, group)
     (4, 64, 256, 40, 3, False, 4, 64), (4, 40, 128, 33, 2, False, 8, 32),
     (8, 64, 256, 1, 100, True, 4, 64), (8, 64, 256, 1, 20, True, 8, 128),
     (16, 48, 192, 1, 70, True, 4, 32), (32, 128, 1024, 2, 300, False, 4, 64),
+    (8, 64, 512, 1, 20, False, 2, 64), (4, 48, 1024, 3, 30, True, 2, 128),
 ]
 
 
