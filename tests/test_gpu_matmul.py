@@ -235,6 +235,22 @@ def test_switch_glu_prefill(gpu_lib, kernel, T, mode):
                      want.reshape(T * d["top_k"], -1))
 
 
+@pytest.mark.parametrize("T,group", [(4, 64), (24, 128)])
+def test_switch_glu_2bit(gpu_lib, T, group):
+    """SwitchGLU with 2-bit codes (hidden 512, intermediate 256, 16 experts, top-2):
+    the fused up/gate and the down launch on the streaming kernel."""
+    q = gpu_lib
+    rng = np.random.default_rng(T + group)
+    E, H, I, top_k = 16, 512, 256, 2
+    up, gate, down = (random_qweight(rng, E, n, k, group, 2) for n, k in ((I, H), (I, H), (H, I)))
+    x = normal_bf16(rng, (T, H))
+    idx = np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.uint32)
+    W = [qweight(*t, group, 2) for t in (up, gate, down)]
+    y = q.qmoe_switch_glu(dev_bf16(x), dev_u32(idx), *W, mode=0)
+    want, _ = O.switch_glu(x, idx, (*up, group, 2), (*gate, group, 2), (*down, group, 2))
+    assert_close(f"switch_glu 2-bit T={T} g{group}", y, want)
+
+
 @pytest.mark.parametrize("T", [40, 331])
 def test_switch_glu_prefill_8bit_g128(gpu_lib, kernel, T):
     """8-bit group-128 prefill SwitchGLU with Zipf-skewed routing: the down projection's
