@@ -72,7 +72,9 @@ static_assert(kKC == 64 || kKC == 128, "step");
 #define QTS_EPI_COLS 32
 #endif
 constexpr int kS1 = QTS_S1;                      // activation stages
-constexpr int kPK = 256 / kKC;                   // steps per packed-code slot (256 k)
+// steps per packed-code slot (128 bytes of each row: 256 k of 4-bit, 128 k of 8-bit codes)
+template <int BITS>
+__host__ __device__ constexpr int steps_per_slot() { return (1024 / BITS) / kKC; }
 constexpr int kPBytes = kM * 128;                // 16 KB: two boxes of 64 rows x 128 B
 constexpr int kSP = QTS_SP;                      // packed-code slots
 constexpr int kSbGroups = 8;                     // groups per scale/bias box
@@ -88,8 +90,11 @@ constexpr int kASlots = QTS_ASLOTS;              // dequantised A tiles in tenso
 #endif
 constexpr int kDqWarps = QTS_DQ_WARPS;           // 8 or 16
 constexpr int kDqParts = kDqWarps / 4;           // k slices of a step, one per warp of a quarter
-constexpr int kTW = kKC / 8 / kDqParts;          // packed words per dequant thread and step
-static_assert((kDqWarps == 8 || kDqWarps == 16) && kTW % 4 == 0, "dequant split");
+constexpr int kKT = kKC / kDqParts;              // k per dequant thread and step
+// packed words per dequant thread and step
+template <int BITS>
+__host__ __device__ constexpr int thread_words() { return kKT * BITS / 32; }
+static_assert((kDqWarps == 8 || kDqWarps == 16) && thread_words<4>() % 4 == 0, "dequant split");
 constexpr int kDCol0 = kASlots * kACols;         // accumulators after the A tiles
 constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 4, kProdWarp = 4, kMmaWarp = 5, kDqWarp0 = 6;
@@ -125,6 +130,10 @@ struct alignas(64) TsParams {
   int64_t dense_rows;
   int64_t N, K;
   int pair;                 // 1: one stack, a unit is 128 of its channels
+  int sb_groups;            // > 0: a row has fewer than 8 groups; each unit's scales and
+                            // biases ([64 rows][sb_groups] per half) come by 1-D bulk copies
+  const uint16_t* scales[2];
+  const uint16_t* biases[2];
   int vec_store;            // y rows start 16-byte aligned: 8 channels per store
   int tma_store;            // one stack, rows in tile order (no dst_row), vec_store: full
                             // epilogue pieces leave by TMA tensor stores
@@ -157,11 +166,27 @@ __device__ __forceinline__ uint32_t ts_mma_n(uint32_t valid) {
 }
 
 
-template <int GS>
+// 4 packed 8-bit codes -> 4 bf16 of q*s + b (the fp32 fma is exact for a <=8-bit code
+// times a bf16 scale plus a bf16 bias; one rounding to bf16).
+__device__ __forceinline__ uint2 ts_dequant_word8(uint32_t w, float s, float b) {
+  float v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t f = prmt(w, 0x4B000000u, k | (4 << 4) | (4 << 8) | (7 << 12));  // 2^23 + q
+    v[k] = fmaf(__uint_as_float(f) - 8388608.0f, s, b);
+  }
+  return make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+
+template <int BITS, int GS, bool SB_WHOLE>
 __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_constant__ TsParams p) {
-  constexpr int KS_SB = kSbGroups * GS / kKC;  // steps per scale/bias window
-  static_assert((kSbGroups * GS) % kKC == 0 && KS_SB >= 1, "group size");
-  constexpr int GPT = (kTW * 8) >= GS ? (kTW * 8) / GS : 1;  // groups of a thread's k per step
+  constexpr int kPK = steps_per_slot<BITS>();
+  constexpr int kTW = thread_words<BITS>();
+  static_assert(kPK >= 1 && kTW % 4 == 0, "code slots");
+  // steps per scale/bias window: 8 groups by TMA, or the whole unit's groups
+  constexpr int KS_SB_BOX = kSbGroups * GS / kKC;
+  static_assert((kSbGroups * GS) % kKC == 0 && KS_SB_BOX >= 1, "group size");
+  constexpr int GPT = kKT >= GS ? kKT / GS : 1;  // groups of a thread's k per step
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -224,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
   if (threadIdx.x == 0) prof_start(p.prof);
 
   const int64_t KS = p.K / kKC;               // steps per unit
+  const int64_t KS_SB = SB_WHOLE ? KS : KS_SB_BOX;
   const int unit_n = p.pair ? kM : kM / 2;    // output channels per unit
   const int64_t NB = (p.N + unit_n - 1) / unit_n;
   const int64_t ntiles = p.dense_rows > 0 ? (p.dense_rows + kNMax - 1) / kNMax : *p.num_tiles;
@@ -301,14 +327,29 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
           if (ks % KS_SB == 0) {
             const uint32_t e = sbit % kSbSlots;
             if (!mbar_wait(&empty_sb[e], ((sbit / kSbSlots) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
-            mbar_arrive_expect_tx(&full_sb[e], kSbBytes);
-            const int32_t gx = static_cast<int32_t>(ks * kKC / GS);
+            if constexpr (SB_WHOLE) {
+              // [64 rows][sb_groups] of each half is contiguous: one bulk copy per array
+              const uint32_t bytes = static_cast<uint32_t>(64 * p.sb_groups * 2);
+              mbar_arrive_expect_tx(&full_sb[e], 4 * bytes);
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+              for (int m = 0; m < 2; ++m)
 #pragma unroll
-              for (int arr = 0; arr < 2; ++arr)
-                tma_load_2d(smem + kOffSb + e * kSbBytes + (m * 2 + arr) * 64 * kSbGroups * 2,
-                            &p.tm_sb[m][arr], &full_sb[e], gx, static_cast<int32_t>(m ? r1 : r0));
+                for (int arr = 0; arr < 2; ++arr) {
+                  const uint16_t* src = (arr ? p.biases[p.pair ? 0 : m] : p.scales[p.pair ? 0 : m]) +
+                                        (m ? r1 : r0) * p.sb_groups;
+                  bulk_load(smem + kOffSb + e * kSbBytes + (m * 2 + arr) * 64 * kSbGroups * 2, src,
+                            bytes, &full_sb[e]);
+                }
+            } else {
+              mbar_arrive_expect_tx(&full_sb[e], kSbBytes);
+              const int32_t gx = static_cast<int32_t>(ks * kKC / GS);
+#pragma unroll
+              for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int arr = 0; arr < 2; ++arr)
+                  tma_load_2d(smem + kOffSb + e * kSbBytes + (m * 2 + arr) * 64 * kSbGroups * 2,
+                              &p.tm_sb[m][arr], &full_sb[e], gx, static_cast<int32_t>(m ? r1 : r0));
+            }
             ++sbit;
           }
         }
@@ -398,31 +439,61 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
         // this thread's kTW words of the row: 16-byte pieces of the slot's 128-byte row,
         // piece c at c ^ (rr & 7)
         const uint8_t* rowp = smem + kOffP + sp * kPBytes + m * 64 * 128 + rr * 128;
-        // the thread's k lie in GPT groups, the first at g0 of the scale window
-        const int g0 = (static_cast<int>((ks * kKC) % (kSbGroups * GS)) + part * (kTW * 8)) / GS;
+        // the thread's k lie in GPT groups, the first at g0 of the scale window (row
+        // stride: 8 groups per TMA window, or the row's sb_groups for whole-unit copies)
+        const int sbs = SB_WHOLE ? p.sb_groups : kSbGroups;
+        const int g0 = SB_WHOLE
+                           ? static_cast<int>((ks * kKC + part * kKT) / GS)
+                           : (static_cast<int>((ks * kKC) % (kSbGroups * GS)) + part * kKT) / GS;
         const uint16_t* sbw = reinterpret_cast<const uint16_t*>(smem + kOffSb + e * kSbBytes);
-        __nv_bfloat162 s2[GPT], b2[GPT];
-        load_group_pairs<GPT>(sbw + (m * 2 * 64 + rr) * kSbGroups + g0, s2);
-        load_group_pairs<GPT>(sbw + ((m * 2 + 1) * 64 + rr) * kSbGroups + g0, b2);
-        uint32_t out[kTW * 4];
+        // the four [64 rows][sbs] arrays sit 64 x 8 elements apart
+        const uint16_t* srow = sbw + (m * 2) * 64 * kSbGroups + rr * sbs + g0;
+        const uint16_t* brow = sbw + (m * 2 + 1) * 64 * kSbGroups + rr * sbs + g0;
+        constexpr int kPieceStep = kKC * BITS / 128;  // 16-byte pieces of a row per step
+        uint32_t out[kKT / 2];                         // two bf16 of consecutive k per column
+        if constexpr (BITS == 4) {
+          __nv_bfloat162 s2[GPT], b2[GPT];
+          load_group_pairs<GPT>(srow, s2);
+          load_group_pairs<GPT>(brow, b2);
 #pragma unroll
-        for (int q = 0; q < kTW / 4; ++q) {
-          const int piece = static_cast<int>(ks % kPK) * (kKC / 32) + part * (kTW / 4) + q;
-          const uint4 pw = *reinterpret_cast<const uint4*>(rowp + ((piece ^ (rr & 7)) << 4));
-          const uint32_t w4[4] = {pw.x, pw.y, pw.z, pw.w};
+          for (int q = 0; q < kTW / 4; ++q) {
+            const int piece = static_cast<int>(ks % kPK) * kPieceStep + part * (kTW / 4) + q;
+            const uint4 pw = *reinterpret_cast<const uint4*>(rowp + ((piece ^ (rr & 7)) << 4));
+            const uint32_t w4[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int gi = ((4 * q + j) * 8) / GS;  // the word's group among the thread's
-            const uint4 v = dequant_word4(w4[j], s2[gi], b2[gi]);
-            out[(4 * q + j) * 4 + 0] = v.x;
-            out[(4 * q + j) * 4 + 1] = v.y;
-            out[(4 * q + j) * 4 + 2] = v.z;
-            out[(4 * q + j) * 4 + 3] = v.w;
+            for (int j = 0; j < 4; ++j) {
+              const int gi = ((4 * q + j) * 8) / GS;  // the word's group among the thread's
+              const uint4 v = dequant_word4(w4[j], s2[gi], b2[gi]);
+              out[(4 * q + j) * 4 + 0] = v.x;
+              out[(4 * q + j) * 4 + 1] = v.y;
+              out[(4 * q + j) * 4 + 2] = v.z;
+              out[(4 * q + j) * 4 + 3] = v.w;
+            }
+          }
+        } else {
+          float sf[GPT], bf[GPT];
+#pragma unroll
+          for (int i = 0; i < GPT; ++i) {
+            sf[i] = bf16_to_f32(srow[i]);
+            bf[i] = bf16_to_f32(brow[i]);
+          }
+#pragma unroll
+          for (int q = 0; q < kTW / 4; ++q) {
+            const int piece = static_cast<int>(ks % kPK) * kPieceStep + part * (kTW / 4) + q;
+            const uint4 pw = *reinterpret_cast<const uint4*>(rowp + ((piece ^ (rr & 7)) << 4));
+            const uint32_t w4[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int gi = ((4 * q + j) * 4) / GS;  // 4 codes per 8-bit word
+              const uint2 v = ts_dequant_word8(w4[j], sf[gi], bf[gi]);
+              out[(4 * q + j) * 2 + 0] = v.x;
+              out[(4 * q + j) * 2 + 1] = v.y;
+            }
           }
         }
-        // A tile: lane r, columns part*kTW*4.. (two bf16 of consecutive k per column)
+        // A tile: lane r, columns part*kKT/2.. (two bf16 of consecutive k per column)
         tmem_st_cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + as * kACols +
-                         part * (kTW * 4), out);
+                         part * (kKT / 2), out);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -555,9 +626,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_ts_kernel(const __grid_consta
   if (threadIdx.x == 0) prof_end(p.prof);
 }
 
-template <int GS>
+template <int BITS, int GS, bool SB_WHOLE>
 cudaError_t launch_ts_gs(const TsParams& prm, cudaStream_t stream) {
-  auto kern = qmm_ts_kernel<GS>;
+  auto kern = qmm_ts_kernel<BITS, GS, SB_WHOLE>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -576,9 +647,21 @@ cudaError_t launch_ts_gs(const TsParams& prm, cudaStream_t stream) {
 }  // namespace
 
 bool qmm_ts_supported(const GemmArgs& a) {
-  if (a.bits != 4 || (a.group != 32 && a.group != 64 && a.group != 128)) return false;
+  if ((a.bits != 4 && a.bits != 8) || (a.group != 32 && a.group != 64 && a.group != 128))
+    return false;
   if (a.K % kKC != 0) return false;                    // whole steps of activation boxes
-  if ((a.K / a.group) % kSbGroups != 0) return false;  // scale/bias rows: 16-byte pitch
+  const int64_t gpr = a.K / a.group;
+  if (gpr % kSbGroups != 0) {
+    // Fewer than 8 groups per row: each unit's scale/bias blocks come by 1-D bulk copies
+    // of whole 64-row halves, which must stay inside the stack (no bounds check) and
+    // start 16-byte aligned.
+    if (gpr >= kSbGroups) return false;
+    if (a.N % (a.nmat == 2 ? 64 : 128) != 0) return false;
+    for (int m = 0; m < a.nmat; ++m)
+      if (reinterpret_cast<uintptr_t>(a.w[m].scales) % 16 != 0 ||
+          reinterpret_cast<uintptr_t>(a.w[m].biases) % 16 != 0)
+        return false;
+  }
   if (a.x_rows <= 0 || a.src_row != nullptr) return false;  // activations in tile order
   return true;
 }
@@ -593,12 +676,14 @@ cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream) {
                           /*swizzle128=*/true);
     if (e != cudaSuccess) return e;
   }
-  const int64_t words = a.K / 8;
+  const int64_t words = a.K * a.bits / 32;
   const int64_t gpr = a.K / a.group;
+  const bool whole = gpr % kSbGroups != 0;  // scales/biases by bulk copies (no tensor map)
   for (int m = 0; m < 2; ++m) {
     const QWeight& wm = a.w[a.nmat == 2 ? m : 0];
     e = make_tmap_2d_u32(&prm.tm_w[m], wm.codes, words, a.E * a.N, 32, 64, /*swizzle128=*/true);
     if (e != cudaSuccess) return e;
+    if (whole) continue;
     e = make_tmap_2d_bf16(&prm.tm_sb[m][0], wm.scales, gpr, a.E * a.N, kSbGroups, 64, false);
     if (e != cudaSuccess) return e;
     e = make_tmap_2d_bf16(&prm.tm_sb[m][1], wm.biases, gpr, a.E * a.N, kSbGroups, 64, false);
@@ -620,9 +705,19 @@ cudaError_t launch_qmm_ts(const GemmArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   prm.d_status = a.d_status;
-  if (a.group == 32) return launch_ts_gs<32>(prm, stream);
-  if (a.group == 64) return launch_ts_gs<64>(prm, stream);
-  return launch_ts_gs<128>(prm, stream);
+  prm.sb_groups = whole ? static_cast<int>(gpr) : 0;
+  for (int m = 0; m < 2; ++m) {
+    prm.scales[m] = a.w[a.nmat == 2 ? m : 0].scales;
+    prm.biases[m] = a.w[a.nmat == 2 ? m : 0].biases;
+  }
+  if (a.bits == 4) {
+    if (a.group == 32) return whole ? launch_ts_gs<4, 32, true>(prm, stream) : launch_ts_gs<4, 32, false>(prm, stream);
+    if (a.group == 64) return whole ? launch_ts_gs<4, 64, true>(prm, stream) : launch_ts_gs<4, 64, false>(prm, stream);
+    return whole ? launch_ts_gs<4, 128, true>(prm, stream) : launch_ts_gs<4, 128, false>(prm, stream);
+  }
+  if (a.group == 32) return whole ? launch_ts_gs<8, 32, true>(prm, stream) : launch_ts_gs<8, 32, false>(prm, stream);
+  if (a.group == 64) return whole ? launch_ts_gs<8, 64, true>(prm, stream) : launch_ts_gs<8, 64, false>(prm, stream);
+  return whole ? launch_ts_gs<8, 128, true>(prm, stream) : launch_ts_gs<8, 128, false>(prm, stream);
 }
 
 }  // namespace qmoe
