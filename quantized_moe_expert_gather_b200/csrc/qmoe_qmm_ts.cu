@@ -9,8 +9,8 @@
 //
 // Roles are those of a weight-stationary tile: a unit is 128 weight rows (64 channels of
 // both stacks, or 128 channels of one) against one tile of up to 192 routed rows of one
-// expert.  The weight rows are dequantised (q*s + b, one bf16 rounding) straight into
-// tensor memory as the M = 128 A operand; the tile's rows are the N operand, read by the
+// expert.  The weight rows are dequantised (q*s + b, one bf16 rounding; 4- or 8-bit codes)
+// straight into tensor memory as the M = 128 A operand; the tile's rows are the N operand, read by the
 // MMA from 128B-swizzled shared memory; N is the tile's valid row count rounded up to
 // 16, so a sparsely routed expert costs MMA work in proportion to its rows.  Against a
 // kernel that stages dequantised weights in shared memory, this halves the
@@ -21,16 +21,20 @@
 // One persistent CTA per SM takes every gridDim-th unit.  Warps:
 //   0-3, 15-18  epilogue, two groups taking alternate pieces: tcgen05.ld of the unit's
 //         128 x N fp32 accumulator in 32-column pieces (one TMEM lane per weight row),
-//         transposed through shared memory into 16-byte stores of 8 output channels
-//         (after silu*mul for two stacks) per valid routed row;
+//         transposed through shared memory; a full piece of one stack in tile order leaves
+//         by one TMA tensor store, others by 16-byte stores of 8 output channels (after
+//         silu*mul for two stacks) per valid routed row;
 //   4     activation producer: TMA of the activation slab of each 128-k step (per 64-k
-//         swizzle atom one box of 64, 128 or 192 rows x 128 B: as many rows as the tile's
-//         MMA N reads);
+//         swizzle atom one box of as many 32-row blocks as the tile's MMA N reads);
 //   5     MMA issuer: tcgen05.mma kind::f16, A from tensor memory, M=128, N <= 192, K=16;
 //   6-13  dequant: warp w owns the weight rows of TMEM lane quarter w%4 and one half of
-//         each step's 128 k (eight packed words per thread and step);
-//   14    weight producer: TMA of the packed codes every 256 k (two boxes of 64 rows x
-//         128 B) and of the scales and biases every 8 groups.
+//         each step's 128 k (64 codes per thread and step);
+//   14    weight producer: TMA of the packed codes per 128 bytes of each row (two boxes of
+//         64 rows x 128 B: 256 k of 4-bit, 128 k of 8-bit codes) and of the scales and
+//         biases every 8 groups -- or, when a row has fewer than 8 groups, the unit's
+//         whole [64 rows][groups] blocks by 1-D bulk copies.  With a tile table written
+//         before the previous kernel (the down projection), the weight producer and the
+//         dequant warps start before that kernel completes.
 // Tensor memory: two 128-k A slots (128 columns) and two 192-column accumulators.  Steps
 // of 128 k rather than 64 halve the mbarrier hand-offs between the roles per flop, which
 // bound the kernel (64-k steps: T=16384 up/gate 684 TFLOP/s; 128-k steps: 885).
