@@ -33,6 +33,13 @@
  *     and stream bit i in bit (i mod 32) of word i/32 -- for 4 and 8 bits, code j of a
  *     word in bits [(j mod 32/bits)*bits, ...); 3-, 5- and 6-bit codes may straddle two
  *     words -- so W [rows, K] packs to [rows, K*bits/32].
+ *   - Kernel choice (results agree within the bf16 tolerance whichever runs): the matmul
+ *     calls plan from the most routed rows one expert can receive -- up to 16 a streaming
+ *     kernel, beyond a tensor-core kernel.  Environment overrides, read at every call:
+ *     QMOE_FORCE_KERNEL=qmv|tc pins the plan; QMOE_PREFILL=tc uses the tensor-core kernel
+ *     that stages weights in shared memory instead of the one that keeps them in tensor
+ *     memory; QMOE_DECODE=qdec runs the streaming plan on the tensor cores; QMOE_PDL=0
+ *     (read once) launches without programmatic dependent launch.
  */
 #ifndef QMOE_H_
 #define QMOE_H_
