@@ -12,10 +12,11 @@ matmul, activation and sum.  See ``qmoe_oracle`` for the per-function citations.
 Parity status of each function (what pins it, in ``tests/test_oracle_*.py``):
 
 * ``bf16_from_f32`` / ``f32_from_bf16``   pinned: hand-computed bit patterns.
-* ``pack_codes`` / ``unpack_codes``       pinned: hand-computed words, round trip.
+* ``pack_codes`` / ``unpack_codes``       pinned: hand-computed words for 1-8-bit codes
+                                          (straddling 3/5/6-bit codes included), round trip.
 * ``quantize`` / ``dequantize``           pinned: the error bounds and constructed
-                                          groups of nuvec-core's quantized.rs tests,
-                                          hand-worked groups.
+                                          groups of nuvec-core's quantized.rs tests over
+                                          every width it tests, hand-worked groups.
 * ``qmm`` / ``gather_qmm``                pinned: exact rational arithmetic
                                           (``fractions``) on tiny shapes, per-batch
                                           selection identity, sorted == unsorted.
