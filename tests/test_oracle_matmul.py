@@ -33,7 +33,9 @@ def _exact_dot(xrow, wrow):
 
 def test_qmm_matches_exact_rational_brute_force():
     rng = np.random.default_rng(0x52)
-    for bits, group in [(4, 32), (8, 64), (4, 128)]:
+    # the (bits, group) pairs of nuvec-core's quantized_matmul_equals_the_dequantized_product
+    for bits, group in [(4, 64), (3, 32), (8, 128), (2, 32), (6, 64), (5, 32), (1, 64),
+                        (4, 32), (8, 64), (4, 128)]:
         N, K, M = 3, 128, 2
         packed, s, b, exact = _dyadic_weight(rng, 1, N, K, group, bits)
         x = bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
