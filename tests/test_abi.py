@@ -53,6 +53,9 @@ def test_quantize_rejects_bad_arguments_on_host(lib):
     fake = 1 << 20  # never dereferenced: validation fails first
     assert lib.qmoe_quantize(fake, 1, 2, 64, 48, 4, fake, fake, fake, None) == ERR_UNSUPPORTED
     assert lib.qmoe_quantize(fake, 1, 2, 64, 64, 7, fake, fake, fake, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_quantize(fake, 1, 2, 64, 64, 0, fake, fake, fake, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_quantize(fake, 1, 2, 64, 64, 9, fake, fake, fake, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_dequantize(fake, fake, fake, 1, 2, 64, 64, 7, fake, 1, None) == ERR_UNSUPPORTED
     assert lib.qmoe_quantize(fake, 1, 2, 96, 64, 4, fake, fake, fake, None) == ERR_ARG
     assert lib.qmoe_quantize(fake, 5, 2, 64, 64, 4, fake, fake, fake, None) == ERR_DTYPE
     assert lib.qmoe_quantize(fake, 1, 0, 64, 64, 4, None, None, None, None) == 0  # empty
@@ -66,6 +69,9 @@ def test_matmuls_reject_bad_arguments_on_host(lib):
     # unsupported codec
     assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 96, 48, 4, fake, None, None) == ERR_UNSUPPORTED
     assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 96, 32, 3, fake, None, None) == ERR_UNSUPPORTED
+    # 2-bit matmuls need groups of 64 or 128; 1-bit codes have no matmul kernel
+    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 64, 32, 2, fake, None, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 64, 64, 1, fake, None, None) == ERR_UNSUPPORTED
     assert lib.qmoe_qmm(fake, 0, fake, fake, fake, 8, 64, 64, 4, fake, None, None) == 0
     # gather: workspace too small
     need = lib.qmoe_gather_qmm_workspace_size(4, 1, 8, 16, 64)
