@@ -107,7 +107,7 @@ def test_tile_table_worked_example(gpu_lib):
     assert host_u32(tiles)[:n].tolist() == g["aligned_tiles"]
 
 
-@pytest.mark.parametrize("bm", [8, 16, 128])
+@pytest.mark.parametrize("bm", [8, 16, 128, 192])
 def test_tile_table_random_bit_exact(gpu_lib, bm):
     q = gpu_lib
     rng = np.random.default_rng(bm)
