@@ -251,6 +251,30 @@ def test_switch_glu_2bit(gpu_lib, T, group):
     assert_close(f"switch_glu 2-bit T={T} g{group}", y, want)
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+def test_switch_glu_prefill_rows_of_few_groups(gpu_lib, bits):
+    """Prefill SwitchGLU whose up/gate rows (hidden 512, group 128) and down rows
+    (intermediate 256) hold fewer than 8 groups: the tensor-memory kernel takes both
+    projections' scales and biases by whole-unit bulk copies (two stacks, then one)."""
+    q = gpu_lib
+    rng = np.random.default_rng(bits)
+    E, H, I, T, top_k, group = 4, 512, 256, 96, 2, 128
+    up, gate, down = (random_qweight(rng, E, n, k, group, bits) for n, k in ((I, H), (I, H), (H, I)))
+    x = normal_bf16(rng, (T, H))
+    idx = np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.uint32)
+    W = [qweight(*t, group, bits) for t in (up, gate, down)]
+    slots = torch.zeros(16 * 16, dtype=torch.uint8, device="cuda")
+    q.qmoe_timing_enable(slots)
+    try:
+        y = q.qmoe_switch_glu(dev_bf16(x), dev_u32(idx), *W, mode=0)
+        torch.cuda.synchronize()
+        assert q.qmoe_timing_read("ts_glu")[1] == 1 and q.qmoe_timing_read("ts")[1] == 1
+    finally:
+        q.qmoe_timing_enable(None)
+    want, _ = O.switch_glu(x, idx, (*up, group, bits), (*gate, group, bits), (*down, group, bits))
+    assert_close(f"switch_glu {bits}-bit g{group} few groups", y, want)
+
+
 @pytest.mark.parametrize("T", [40, 331])
 def test_switch_glu_prefill_8bit_g128(gpu_lib, kernel, T):
     """8-bit group-128 prefill SwitchGLU with Zipf-skewed routing: the down projection's
