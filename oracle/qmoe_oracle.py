@@ -29,13 +29,33 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "CODE_BITS", "bf16_from_f32", "f32_from_bf16", "pack_codes", "unpack_codes", "quantize",
+    "CODE_BITS", "bf16_from_f32", "bf16_from_f64", "f32_from_bf16", "pack_codes", "unpack_codes", "quantize",
     "dequantize", "qmm", "gather_qmm", "gather_mm", "sort_by_expert", "tile_table",
     "silu", "switch_glu", "moe_combine", "moe_combine_stock", "sigmoid",
 ]
 
 
 # ----------------------------------------------------------------------------- bf16
+
+def bf16_from_f64(v: np.ndarray) -> np.ndarray:
+    """float64 -> bf16 bit patterns rounded ONCE to nearest, ties to even (finite
+    inputs).
+
+    The value is first rounded to float32 with round-to-odd (truncate toward zero,
+    then set the last significand bit when anything was dropped) and that float32 is
+    rounded to bf16 to nearest-even.  Round-to-odd at 24 bits keeps every bit the
+    second rounding to 8 bits needs, so the result equals one direct rounding of the
+    float64 value; plain float32 rounding first would double-round (1 + 2^-8 + 2^-30
+    would land on the tie 1 + 2^-8 and go down to 1 instead of up to 1 + 2^-7).
+    """
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    f = v.astype(np.float32)
+    too_big = np.abs(f.astype(np.float64)) > np.abs(v)
+    f = np.where(too_big, np.nextafter(f, np.float32(0)), f).astype(np.float32)
+    inexact = f.astype(np.float64) != v
+    u = f.view(np.uint32) | np.where(inexact, np.uint32(1), np.uint32(0))
+    return bf16_from_f32(u.view(np.float32))
+
 
 def f32_from_bf16(u16: np.ndarray) -> np.ndarray:
     """bf16 bit patterns -> float32 values (exact: bf16 is the top half of fp32)."""
@@ -85,8 +105,17 @@ def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
 
 
 def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
-    """Inverse of :func:`pack_codes`; returns int64 codes."""
+    """Inverse of :func:`pack_codes`; returns int64 codes.
+
+    For widths that divide 32 no code straddles a word, so code j of a word is
+    simply ``(word >> (j*bits)) & (2^bits - 1)``; other widths walk the bit stream.
+    """
     assert bits in CODE_BITS
+    if 32 % bits == 0:
+        w = np.asarray(words, dtype=np.uint32)
+        shifts = (np.arange(32 // bits, dtype=np.uint32) * np.uint32(bits))
+        codes = (w[..., :, None] >> shifts) & np.uint32((1 << bits) - 1)
+        return codes.reshape(w.shape[:-1] + (-1,)).astype(np.int64)
     w = np.asarray(words, dtype=np.uint64)
     stream = (w[..., :, None] >> np.arange(32, dtype=np.uint64)) & np.uint64(1)
     stream = stream.reshape(w.shape[:-1] + (-1,))
@@ -320,8 +349,10 @@ def switch_glu(x, indices, up, gate, down):
 
     ``x``: bf16 ``[T, H]``; ``indices``: ``[T, top_k]``; each weight is a tuple
     ``(packed [E,N,K*bits/32], scales, biases, group, bits)``.  u and g are fp64;
-    h is rounded to bf16 once (it is the bf16 input of the down projection); y is
-    fp64.  Returns ``(y [T, top_k, H], h_bits [T, top_k, I])``.
+    h is rounded from fp64 to bf16 once (it is the bf16 input of the down
+    projection); y is fp64.  The rows routed to one expert go through its three
+    matrices together (one fp64 matrix product per matrix).  Returns
+    ``(y [T, top_k, H], h_bits [T, top_k, I])``.
     """
     idx = np.asarray(indices, np.int64)
     T, top_k = idx.shape
@@ -337,12 +368,13 @@ def switch_glu(x, indices, up, gate, down):
     h_bits = np.empty((T, top_k, inter), np.uint16)
     for e in np.unique(idx):  # dequantise each routed expert once
         wu, wg, wd = dq(up, e), dq(gate, e), dq(down, e)
-        for t, k in zip(*np.nonzero(idx == e)):
-            u = wu @ xf[t]
-            g = wg @ xf[t]
-            h = bf16_from_f32((silu(g) * u).astype(np.float32))
-            h_bits[t, k] = h
-            y[t, k] = wd @ f32_from_bf16(h).astype(np.float64)
+        ts, ks = np.nonzero(idx == e)
+        xe = xf[ts]                      # [rows, H]
+        u = xe @ wu.T
+        g = xe @ wg.T
+        h = bf16_from_f64(silu(g) * u)
+        h_bits[ts, ks] = h
+        y[ts, ks] = f32_from_bf16(h).astype(np.float64) @ wd.T
     return y, h_bits
 
 

@@ -27,6 +27,32 @@ def test_bf16_round_to_nearest_even_hand_patterns():
     assert O.f32_from_bf16(np.array([0x3F80, 0x4070], np.uint16)).tolist() == [1.0, 3.75]
 
 
+def test_bf16_from_f64_rounds_once():
+    """fp64 -> bf16 is one round-to-nearest-even step (the SwitchGLU's h is rounded
+    to bf16 once).  Hand patterns where rounding through float32 first would differ,
+    then exact-rational nearest-even checks on random values."""
+    from fractions import Fraction
+    v = np.array([1 + 2.0**-8 + 2.0**-30, 1 + 2.0**-8, 1 + 3 * 2.0**-8,
+                  -(1 + 2.0**-8 + 2.0**-40), 0.0, 3.75], np.float64)
+    assert [int(b) for b in O.bf16_from_f64(v)] == [0x3F81, 0x3F80, 0x3F82, 0xBF81, 0x0000,
+                                                      0x4070]
+    rng = np.random.default_rng(11)
+    vals = rng.standard_normal(400) * np.exp2(rng.integers(-60, 60, 400))
+    got = O.bf16_from_f64(vals)
+
+    def val(bits):
+        return Fraction(float(O.f32_from_bf16(np.array([bits], np.uint16))[0]))
+
+    for x, b in zip(vals, got):
+        b = int(b)
+        fx, here = Fraction(float(x)), val(b)
+        for nb in (b - 1, b + 1):  # neighbours with the same sign, magnitude +- 1 ulp
+            if (nb & 0x7FFF) == 0x7F80 or (nb & 0x8000) != (b & 0x8000):
+                continue
+            d0, d1 = abs(fx - here), abs(fx - val(nb))
+            assert d0 < d1 or (d0 == d1 and (b & 1) == 0), (x, hex(b), hex(nb))
+
+
 def test_pack_layout_hand_words():
     assert O.pack_codes(np.arange(8)[None], 4)[0, 0] == 0x76543210
     assert O.pack_codes(np.array([[1, 2, 3, 4]]), 8)[0, 0] == 0x04030201
