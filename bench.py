@@ -246,8 +246,9 @@ def run_reference(args, rank, ws):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": CONFIG,
         "cpu_baseline": {"kind": "oracle", "value": gbs, "unit": "GB/s", "cores": 1,
+                         "nproc": os.cpu_count(), "cores_available": len(os.sched_getaffinity(0)),
                          "sample": "one decode token per step: SwitchGLU over its 8 experts "
-                                   "(113 MB of packed weights) + combine, fp64"},
+                                   "(113 MB of packed weights) + combine, fp64, one thread"},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -323,9 +324,46 @@ def run_prefill(q, token_counts, dev, peaks, reps=5):
         out[f"T{T}"] = {"ms": t, "tflops": tf, "frac_bf16_peak": tf / bf16_peak,
                         "bytes_moved": moved, "gbs": gbs, "frac_hbm": gbs / hbm_peak,
                         "touched_experts": touched,
-                        "kernel_ms": split, "upgate_tflops": glu_tf, "down_tflops": dn_tf}
+                        "upgate_tflops": glu_tf, "down_tflops": dn_tf,
+                        "upgate_ms": glu_ms, "down_ms": dn_ms,
+                        "upgate_kernel": "qmm_ts" if split["ts_glu"] else
+                                         "qmm_tc" if split["tc_glu"] else "qmv",
+                        **{f"{k}_ms": v for k, v in split.items() if v}}
         del Wp, d
     return out
+
+
+def flat(d, sep="_"):
+    """Nested result dicts -> one level of scalar values (keys joined by ``sep``):
+    the form the JSON line's sub-objects keep."""
+    out = {}
+    for k, v in d.items():
+        if isinstance(v, dict):
+            for k2, v2 in flat(v, sep).items():
+                out[f"{k}{sep}{k2}"] = v2
+        else:
+            out[k] = v
+    return out
+
+
+def prefill_roofline(prefill, peaks):
+    """Roofline of the prefill up/gate launch at the largest token count: its FLOP per
+    launch over its live launch time, against the measured bf16 peak."""
+    if not prefill:
+        return None
+    T = max(int(k[1:]) for k in prefill)
+    r = prefill[f"T{T}"]
+    peak = peaks["bf16_tflops"] if peaks else 1590.0
+    flop = T * TOP_K * 4 * 2048 * 512
+    ach = r["upgate_tflops"]
+    return {"kernel": f"{r['upgate_kernel']} up/gate gather_qmm + silu*mul, T={T}",
+            "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+            "frac": ach / peak if ach else None,
+            "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, burst)" if peaks
+                           else "fallback",
+            "flop_per_launch": flop, "launch_us": 1e3 * r["upgate_ms"] if r["upgate_ms"] else None,
+            "traffic": None,
+            "layer_ms": r["ms"], "layer_tflops": r["tflops"], "layer_frac": r["frac_bf16_peak"]}
 
 
 def _graph_time(fn, reps=8):
@@ -638,7 +676,7 @@ def main():
                           "the bytes touched",
         "launch_us": 1e3 * k_ms / k_n if k_n else None,
         "bytes_per_launch": ug_bytes / k_n if k_n else None,
-        "kernel_ms_in_timed_steps": sums, "step_total_ms": ms,
+        **{f"{k}_ms_in_timed_steps": v for k, v in sums.items()}, "step_total_ms": ms,
     }
 
     # end to end through the public API with host buffers (pinned), copies timed
@@ -740,8 +778,10 @@ def main():
                 b_tot += b
                 n += 1
         cpu = {"value": b_tot / t_tot / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "nproc": os.cpu_count(), "cores_available": len(os.sched_getaffinity(0)),
                "sample": f"{n} decode token(s): SwitchGLU over 8 experts + combine in fp64 "
-                         f"({t_tot:.1f} s)"}
+                         f"({t_tot:.1f} s), one thread (BLAS limited to 1) of the host's "
+                         f"{os.cpu_count()}"}
 
     if rank == 0:
         line = {
@@ -750,8 +790,13 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(CONFIG, experts=args.experts), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches,
-            "decode_isolated": isolated, "prefill": prefill, "dense_qmm": dense,
-            "moe_block": block, "combine": combine, "gather_mm_bf16": gmm,
+            "roofline_prefill": prefill_roofline(prefill, peaks),
+            "decode_isolated": flat(isolated),
+            "prefill": flat(prefill) if prefill else None,
+            "dense_qmm": flat(dense) if dense else None,
+            "moe_block": flat(block) if block else None,
+            "combine": flat(combine) if combine else None,
+            "gather_mm_bf16": flat(gmm) if gmm else None,
             "hbm_frac_of_measured": value / hbm_peak,
         }
         print(json.dumps(line), flush=True)

@@ -38,8 +38,7 @@
  *     kernel, beyond a tensor-core kernel.  Environment overrides, read at every call:
  *     QMOE_FORCE_KERNEL=qmv|tc pins the plan; QMOE_PREFILL=tc uses the tensor-core kernel
  *     that stages weights in shared memory instead of the one that keeps them in tensor
- *     memory; QMOE_DECODE=qdec runs the streaming plan on the tensor cores; QMOE_PDL=0
- *     (read once) launches without programmatic dependent launch.
+ *     memory; QMOE_PDL=0 (read once) launches without programmatic dependent launch.
  */
 #ifndef QMOE_H_
 #define QMOE_H_
@@ -75,7 +74,9 @@ enum { QMOE_DTYPE_BF16 = 0, QMOE_DTYPE_F32 = 1 };
 /* Bits OR-ed into *d_status by kernels. */
 enum {
   QMOE_DEV_BAD_INDEX = 1,     /* an expert or row index was out of range; its rows are zero */
-  QMOE_DEV_TIMEOUT = 2        /* a bounded wait ran out; the call's outputs are undefined    */
+  QMOE_DEV_TIMEOUT = 2,       /* a bounded wait ran out; the call's outputs are undefined    */
+  QMOE_DEV_UNSORTED = 4       /* sorted_indices was set but rhs decreases somewhere; the
+                                 result is still correct (rows are sorted by expert anyway) */
 };
 
 /* One quantised weight stack: codes [E, N, K*bits/32] uint32, scales and biases
@@ -87,6 +88,17 @@ typedef struct {
   int64_t E, N, K;
   int32_t group, bits;
 } qmoe_qweight;
+
+/*
+ * qmoe_debug_skip_stage -- test hook of the bounded waits (no page counterpart).  The
+ * next launch of the streaming kernel (qmoe_qmm / qmoe_gather_qmm / qmoe_switch_glu on
+ * few rows per expert) leaves the copies of pipeline stage `stage` of its last CTA
+ * unissued, so the waits for that stage run out: the kernel sets QMOE_DEV_TIMEOUT in
+ * its d_status, stops every role, lets its issued copies land and returns, leaving
+ * its outputs undefined; the next call is unaffected.  A wait runs out after about a
+ * second.  stage < 0 disarms the hook.  Host state, one-shot; returns QMOE_OK.
+ */
+QMOE_API int qmoe_debug_skip_stage(int64_t stage);
 
 /* Human-readable name of a status code (static string; never NULL). */
 QMOE_API const char* qmoe_status_string(int status);
@@ -169,8 +181,9 @@ QMOE_API int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, cons
  *                x_batches == B; one x batch per token over its experts when
  *                B = x_batches*top_k)
  *   rhs_indices  [B] uint32 or NULL: NULL means rhs[b] = b*E/B
- *   sorted_indices  a promise that rhs is non-decreasing; it only selects the kernel
- *                (results are identical either way)
+ *   sorted_indices  a promise that rhs is non-decreasing; results are identical
+ *                either way (the rows are sorted by expert on the device), and a
+ *                broken promise sets QMOE_DEV_UNSORTED
  *   workspace    device scratch of at least qmoe_gather_qmm_workspace_size() bytes
  *   y            [B, M, N] bf16 (out)
  * Rows whose rhs >= E or lhs >= x_batches are written as zeros and flag
@@ -190,14 +203,21 @@ QMOE_API int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, i
  * workspace -- e.g. a plugin that is given only its input and output tensors by a
  * host framework that owns all device memory, or a serving loop that must not call
  * cudaMalloc (it can synchronise the device) between requests.
- *   Arguments as qmoe_gather_qmm, without the workspace.  The routing metadata lives
- *   in a fixed 128 KiB array in device memory inside the library (one copy per GPU
- *   that loads the library, held until the process exits).  The call allocates
- *   nothing and runs the streaming kernel path.
+ *   Arguments as qmoe_gather_qmm, without the workspace, except that only 4- and
+ *   8-bit codes in groups of 32, 64 or 128 are taken (others: QMOE_ERR_UNSUPPORTED).
+ *   The routing metadata lives in a fixed 128 KiB array in device memory inside the
+ *   library (one copy per GPU that loads the library, held until the process exits).
+ *   The call allocates nothing and runs the streaming kernel at every row count: it
+ *   reads an expert's weights once per tile of 8 or 16 routed rows, so with many rows
+ *   per expert (prefill-sized calls, skewed routing) it re-reads a heavy expert's
+ *   weights up to 256 times and runs far below qmoe_gather_qmm's tensor-core path.
  *   Limits: B*M <= 4096 routed rows and E <= 1024 experts; larger problems return
  *   QMOE_ERR_TOO_LARGE before any launch.
  *   The first call on a device looks up the array's device address (with that device
- *   current); make that first call before any stream capture.
+ *   current); make that first call before any stream capture.  The address is kept
+ *   for the life of the process: after cudaDeviceReset (or anything else that
+ *   destroys the device's primary context) do not call this entry point again in
+ *   that process.
  *   All calls share the array: calls that overlap on the GPU (other streams, other
  *   threads) race on it and must be serialised by the caller.
  */

@@ -24,14 +24,15 @@ __all__ = [
     "qmoe_gather_qmm_workspace_size", "qmoe_gather_qmm_noalloc", "qmoe_sort_by_expert", "qmoe_tile_table",
     "qmoe_switch_glu", "qmoe_switch_glu_workspace_size", "qmoe_moe_combine",
     "qmoe_moe_combine_stock", "qmoe_gather_mm", "qmoe_gather_mm_workspace_size", "QWeight",
-    "QMOE_DEV_BAD_INDEX", "QMOE_DEV_TIMEOUT", "EXPORTED",
+    "QMOE_DEV_BAD_INDEX", "QMOE_DEV_TIMEOUT", "QMOE_DEV_UNSORTED", "qmoe_debug_skip_stage",
+    "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: Optional[ctypes.CDLL] = None
 
 QMOE_DTYPE_BF16, QMOE_DTYPE_F32 = 0, 1
-QMOE_DEV_BAD_INDEX, QMOE_DEV_TIMEOUT = 1, 2
+QMOE_DEV_BAD_INDEX, QMOE_DEV_TIMEOUT, QMOE_DEV_UNSORTED = 1, 2, 4
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -47,6 +48,7 @@ class _QWeight(ctypes.Structure):
 # name -> (restype, argtypes); the exact list of symbols include/qmoe.h declares.
 _SIGS = {
     "qmoe_status_string": (ctypes.c_char_p, [_i32]),
+    "qmoe_debug_skip_stage": (_i32, [_i64]),
     "qmoe_launch_count": (ctypes.c_uint64, []),
     "qmoe_timing_enable": (_i32, [_p, _i64]),
     "qmoe_timing_read": (_i32, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -136,6 +138,13 @@ _BF16 = (torch.bfloat16,)
 
 def qmoe_status_string(status: int) -> str:
     return load().qmoe_status_string(status).decode()
+
+
+def qmoe_debug_skip_stage(stage: int) -> None:
+    """Test hook of the bounded waits: the next streaming-kernel launch leaves pipeline
+    stage ``stage`` of its last CTA unissued (its waits run out, QMOE_DEV_TIMEOUT);
+    a negative stage disarms it."""
+    _check("qmoe_debug_skip_stage", load().qmoe_debug_skip_stage(stage))
 
 
 def qmoe_launch_count() -> int:
@@ -243,17 +252,27 @@ def qmoe_gather_qmm_noalloc(x, codes, scales, biases, lhs_indices=None, rhs_indi
                             out=None, status=None):
     """As :func:`qmoe_gather_qmm`, for callers that cannot allocate device scratch:
     the library keeps the routing metadata in its own fixed device array (B*M <= 4096,
-    E <= 1024; overlapping calls race on it).  Pass ``out`` to allocate nothing here."""
+    E <= 1024; overlapping calls race on it).  4- and 8-bit codes in groups of 32, 64
+    or 128; it runs the streaming kernel at every row count.  Pass ``out`` to
+    allocate nothing here."""
     _need(x, "x", _BF16)
     _need(codes, "codes", _CODES)
     xb, M, K = x.shape
     E, N = codes.shape[0], codes.shape[1]
+    if lhs_indices is not None:
+        _need(lhs_indices, "lhs_indices", _IDX)
+    if rhs_indices is not None:
+        _need(rhs_indices, "rhs_indices", _IDX)
     if rhs_indices is not None:
         B = rhs_indices.numel()
     elif lhs_indices is not None:
         B = lhs_indices.numel()
     else:
         B = max(xb, E)
+    if lhs_indices is not None and lhs_indices.numel() != B:
+        raise ValueError("lhs_indices and rhs_indices have different sizes")
+    if out is not None:
+        _need(out, "out", _BF16, (B, M, N))
     y = out if out is not None else torch.empty((B, M, N), dtype=torch.bfloat16, device=x.device)
     _check("qmoe_gather_qmm_noalloc", load().qmoe_gather_qmm_noalloc(
         _ptr(x), xb, M, K, _ptr(codes), _ptr(scales), _ptr(biases), E, N, group, bits,

@@ -74,7 +74,6 @@ constexpr int kTcBm = 128;
 struct Plan {
   bool tc;
   int bm;
-  bool qdec = false;  // streaming on the tensor cores (tiles of 16 rows, rows gathered first)
   bool ts = false;    // tensor cores with the weights in tensor memory (tiles of 192 rows)
 };
 // QMOE_PREFILL=tc keeps the tensor-core plan on the kernel that stages dequantised
@@ -83,20 +82,13 @@ bool ts_allowed() {
   const char* v = std::getenv("QMOE_PREFILL");
   return v == nullptr || std::strcmp(v, "tc") != 0;
 }
-// The streaming kernel on the tensor cores (QMOE_DECODE=qdec) instead of mma.sync.
-bool qdec_requested() {
-  const char* v = std::getenv("QMOE_DECODE");
-  return v != nullptr && std::strcmp(v, "qdec") == 0;
-}
-Plan plan_for(int64_t R, int64_t E, int64_t max_rows, bool tc_ok, bool qdec_ok = false,
-              bool ts_ok = false) {
+Plan plan_for(int64_t R, int64_t E, int64_t max_rows, bool tc_ok, bool ts_ok = false) {
   const Kernel k = forced_kernel();
   const int64_t touched = std::max<int64_t>(1, std::min(E, R));
   Plan stream{false, R / touched > 8 ? 16 : 8};
-  if (qdec_ok && qdec_requested()) stream = Plan{false, 16, true};
   if (!(tc_ok || ts_ok) || k == Kernel::Qmv) return stream;
   if (k == Kernel::Tc || max_rows > 16) {
-    if (ts_ok && ts_allowed()) return Plan{true, kTsTileRows, false, true};
+    if (ts_ok && ts_allowed()) return Plan{true, kTsTileRows, true};
     if (tc_ok) return Plan{true, kTcBm};
   }
   return stream;
@@ -208,12 +200,10 @@ int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, const qmoe_bf
   const bool big = k == Kernel::Tc || (k == Kernel::Auto && M >= 32);
   const bool ts = big && ts_allowed() && qmm_ts_supported(a);
   const bool tc = !ts && big && qmm_tc_supported(a);
-  const bool qdec = !ts && !tc && qdec_requested() && qdec_supported(a);
-  a.bm = ts ? kTsTileRows : tc ? kTcBm : (qdec || M > 8 ? 16 : 8);
+  a.bm = ts ? kTsTileRows : tc ? kTcBm : (M > 8 ? 16 : 8);
   a.max_tiles = (M + a.bm - 1) / a.bm;
   auto s = static_cast<cudaStream_t>(stream);
   if (ts) return cuda_status(launch_qmm_ts(a, s));
-  if (qdec) return cuda_status(launch_qdec(a, s));
   return cuda_status(tc ? launch_qmm_tc(a, s) : launch_qmv(a, s));
 }
 
@@ -231,7 +221,8 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
                     int64_t E, int64_t N, int group, int bits, const uint32_t* lhs_indices,
                     const uint32_t* rhs_indices, int64_t B, int sorted_indices, void* workspace,
                     size_t workspace_bytes, qmoe_bf16* y, int* d_status, qmoe_stream stream) {
-  (void)sorted_indices;  // a promise about rhs; the expert sort makes it unnecessary
+  // sorted_indices is a promise about rhs: the expert sort makes the result independent
+  // of it; a broken promise is flagged (QMOE_DEV_UNSORTED).
   const int c = check_codec(K, group, bits);
   if (c != QMOE_OK) return c;
   if (x_batches <= 0 || M < 0 || B < 0 || E <= 0 || N <= 0) return QMOE_ERR_ARG;
@@ -265,7 +256,7 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   GemmArgs a_sorted = a;  // as the tensor-core streaming kernel would read x
   a_sorted.x = x_sorted;
   a_sorted.src_row = nullptr;
-  const Plan pl = plan_for(R, E, R > kTcBm ? R : 16, qmm_tc_supported(a), qdec_supported(a_sorted),
+  const Plan pl = plan_for(R, E, R > kTcBm ? R : 16, qmm_tc_supported(a),
                            qmm_ts_supported(a_sorted));
   a.bm = pl.bm;
   a.max_tiles = max_tiles_for(R, E, pl.bm);
@@ -288,6 +279,7 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
   ra.zero_out = y;
   ra.zero_cols = N;
   ra.zero_by_pos = false;
+  ra.check_sorted = sorted_indices != 0;
   ra.d_status = d_status;
   auto s = static_cast<cudaStream_t>(stream);
   if (launch_route(ra, rb.route_ws, s) != cudaSuccess) return QMOE_ERR_CUDA;
@@ -296,12 +288,6 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
     a.x = x_sorted;  // row tiles over the expert-ordered rows
     a.src_row = nullptr;
     return cuda_status(pl.ts ? launch_qmm_ts(a, s) : launch_qmm_tc(a, s));
-  }
-  if (pl.qdec) {
-    if (launch_gather_rows(x, rb.src_row, R, K, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
-    a.x = x_sorted;
-    a.src_row = nullptr;
-    return cuda_status(launch_qdec(a, s));
   }
   a.x = x;  // the streaming kernel reads x through src_row
   a.src_row = rb.src_row;
@@ -316,7 +302,8 @@ int qmoe_gather_mm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K, 
                    int64_t E, int64_t N, const uint32_t* lhs_indices, const uint32_t* rhs_indices,
                    int64_t B, int sorted_indices, void* workspace, size_t workspace_bytes,
                    qmoe_bf16* y, int* d_status, qmoe_stream stream) {
-  (void)sorted_indices;  // a promise about rhs; the expert sort makes it unnecessary
+  // sorted_indices is a promise about rhs: the expert sort makes the result independent
+  // of it; a broken promise is flagged (QMOE_DEV_UNSORTED).
   if (K <= 0 || x_batches <= 0 || M < 0 || B < 0 || E <= 0 || N <= 0) return QMOE_ERR_ARG;
   if (K % 64 != 0) return QMOE_ERR_UNSUPPORTED;
   if (B == 0 || M == 0) return QMOE_OK;
@@ -365,6 +352,7 @@ int qmoe_gather_mm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K, 
   ra.zero_out = y;
   ra.zero_cols = N;
   ra.zero_by_pos = false;
+  ra.check_sorted = sorted_indices != 0;
   ra.d_status = d_status;
   auto s = static_cast<cudaStream_t>(stream);
   if (launch_route(ra, rb.route_ws, s) != cudaSuccess) return QMOE_ERR_CUDA;
@@ -480,7 +468,6 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   GemmArgs ug_sorted = ug;  // as the tensor-core streaming kernel would read x
   ug_sorted.src_row = nullptr;
   const Plan pl = plan_for(R, E, T, qmm_tc_supported(ug) && qmm_tc_supported(dn),
-                           qdec_supported(ug_sorted) && qdec_supported(dn),
                            qmm_ts_supported(ug_sorted) && qmm_ts_supported(dn));
   ug.bm = dn.bm = pl.bm;
   ug.max_tiles = dn.max_tiles = max_tiles_for(R, E, pl.bm);
@@ -515,13 +502,6 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
     }
     if (launch_qmm_tc(ug, s) != cudaSuccess) return QMOE_ERR_CUDA;
     return cuda_status(launch_qmm_tc(dn, s));
-  }
-  if (pl.qdec) {
-    if (launch_gather_rows(x, rb.src_row, R, H, x_sorted, s) != cudaSuccess) return QMOE_ERR_CUDA;
-    ug.x = x_sorted;
-    ug.src_row = nullptr;
-    if (launch_qdec(ug, s) != cudaSuccess) return QMOE_ERR_CUDA;
-    return cuda_status(launch_qdec(dn, s));
   }
   ug.x = x;
   ug.src_row = rb.src_row;

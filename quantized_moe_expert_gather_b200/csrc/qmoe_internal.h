@@ -83,6 +83,8 @@ struct RouteArgs {
   uint16_t* zero_out = nullptr;
   int64_t zero_cols = 0;
   bool zero_by_pos = false;
+  // The caller promised sorted rhs indices: flag QMOE_DEV_UNSORTED where they decrease.
+  bool check_sorted = false;
   int* d_status = nullptr;
 };
 size_t route_workspace_bytes(int64_t R, int64_t E);
@@ -124,11 +126,10 @@ struct GemmArgs {
   bool tiles_ready = false;
   int* d_status = nullptr;
 };
+// Test hook of the bounded waits (qmoe_debug_skip_stage): the stage the next streaming
+// launch's last CTA leaves unissued, or -1.  Read and cleared by that launch.
+int64_t take_skip_stage();
 cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream);   // tiles of <= 16 rows
-// Tensor-core streaming kernel for few rows per expert (tiles of <= 16 rows): 4-bit codes,
-// activations already in tile order (x_rows rows, src_row null).
-bool qdec_supported(const GemmArgs& a);
-cudaError_t launch_qdec(const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream); // tiles of 128 rows
 bool qmm_tc_supported(const GemmArgs& a);
 // Tensor-core kernel with the dequantised weights as the MMA A operand in tensor memory,

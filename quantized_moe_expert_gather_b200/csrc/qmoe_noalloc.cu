@@ -29,7 +29,9 @@ constexpr size_t kScratchBytes = 128 * 1024;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 // Device address of g_noalloc_scratch per device ordinal, looked up once per device
-// with that device current (the first call on a device does it).
+// with that device current (the first call on a device does it).  The address is
+// kept for the life of the process: it is not looked up again after a device reset
+// or anything else that destroys and recreates the device's primary context.
 void* scratch_for_current_device(int* status) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
@@ -76,7 +78,6 @@ extern "C" int qmoe_gather_qmm_noalloc(const qmoe_bf16* x, int64_t x_batches, in
                                        int sorted_indices, qmoe_bf16* y, int* d_status,
                                        qmoe_stream stream) {
   using namespace qmoe;
-  (void)sorted_indices;
   if (!((bits == 4 || bits == 8) && (group == 32 || group == 64 || group == 128)))
     return QMOE_ERR_UNSUPPORTED;
   if (K <= 0 || K % group != 0) return QMOE_ERR_ARG;
@@ -131,6 +132,7 @@ extern "C" int qmoe_gather_qmm_noalloc(const qmoe_bf16* x, int64_t x_batches, in
   ra.zero_out = y;
   ra.zero_cols = N;
   ra.zero_by_pos = false;
+  ra.check_sorted = sorted_indices != 0;
   ra.d_status = d_status;
   auto s = static_cast<cudaStream_t>(stream);
   if (launch_route(ra, route_ws, s) != cudaSuccess) return QMOE_ERR_CUDA;

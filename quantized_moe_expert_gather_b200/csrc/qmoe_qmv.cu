@@ -41,6 +41,7 @@
 //
 // All waits are bounded (see qmoe_common.cuh).
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cudaTypedefs.h>
 #include <mutex>
@@ -121,6 +122,7 @@ struct alignas(64) QmvParams {
   int sb_tma;                   // scales/biases by TMA (row pitch a multiple of 16 bytes)
   int sb_vec;                   // else: byte width of the copy pieces (2: plain copies)
   int early_weights;            // the producer may stream before the previous kernel ends
+  int64_t skip_stage;           // test hook: stage the last CTA leaves unissued (-1: none)
   int* d_status;
   ProfSlot* prof;
 };
@@ -236,6 +238,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
           aborted = true;
           break;
         }
+        // test hook of the bounded waits: nothing lands in this stage, so its waits run out
+        if (blockIdx.x == gridDim.x - 1 && static_cast<int64_t>(it) == p.skip_stage) continue;
         uint8_t* st = smem + stage * C::STAGE_BYTES;
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[stage], C::TMA_BYTES + (p.sb_tma ? C::SB_BYTES : 0u));
@@ -712,6 +716,12 @@ cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cuda
 
 }  // namespace
 
+namespace {
+std::atomic<int64_t> g_skip_stage{-1};
+}  // namespace
+
+int64_t take_skip_stage() { return g_skip_stage.exchange(-1); }
+
 cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
   QmvParams prm{};
   prm.pair = a.nmat == 2 ? 0 : 1;
@@ -728,6 +738,7 @@ cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
   prm.num_tiles = a.num_tiles;
   prm.dense_rows = a.dense_rows;
   prm.early_weights = (a.dense_rows > 0 || a.tiles_ready) ? 1 : 0;
+  prm.skip_stage = take_skip_stage();
   prm.N = a.N;
   prm.K = a.K;
   prm.E = a.E;
@@ -750,3 +761,8 @@ cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace qmoe
+
+extern "C" int qmoe_debug_skip_stage(int64_t stage) {
+  qmoe::g_skip_stage.store(stage < 0 ? -1 : stage);
+  return QMOE_OK;
+}

@@ -40,9 +40,19 @@ struct RouteDev {
   uint16_t* zero_out;
   int64_t zero_cols;
   bool zero_by_pos;
+  bool check_sorted;  // flag rhs indices that decrease (the caller promised sorted ones)
   int* d_status;
   ProfSlot* prof;
 };
+
+// With check_sorted, a batch whose expert index is below the previous batch's breaks
+// the caller's promise of sorted rhs indices: flag it (the result does not depend on
+// the promise, the rows are sorted here anyway).
+__device__ __forceinline__ void check_rhs_order(const RouteDev& d, int64_t r) {
+  if (!d.check_sorted || d.rhs == nullptr || r % d.M != 0) return;
+  const int64_t b = r / d.M;
+  if (b > 0 && d.rhs[b] < d.rhs[b - 1]) set_status(d.d_status, QMOE_DEV_UNSORTED);
+}
 
 // Expert key of routed row r (E for an invalid expert or x row) and its x row.
 __device__ __forceinline__ uint32_t row_key(const RouteDev& d, int64_t r, uint32_t* xrow) {
@@ -64,7 +74,10 @@ __device__ void phase_count(const RouteDev& d, int64_t chunk, uint8_t* cnt) {
   __syncthreads();
   const int64_t r = chunk * kChunk + tid;
   uint32_t key = kNoRow, xrow = 0;
-  if (r < d.R) key = row_key(d, r, &xrow);
+  if (r < d.R) {
+    key = row_key(d, r, &xrow);
+    check_rhs_order(d, r);
+  }
   const uint32_t mask = __match_any_sync(0xFFFFFFFFu, key);
   const uint32_t lt = (1u << lane) - 1u;
   const uint32_t rank = __popc(mask & lt);
@@ -230,7 +243,10 @@ __global__ void __launch_bounds__(kChunk) route_fused_kernel(RouteDev d) {
   for (int64_t i = tid; i < 32 * nb; i += blockDim.x) cnt[i] = 0;
   const int64_t r = tid;
   uint32_t key = kNoRow, xrow = 0;
-  if (r < d.R) key = row_key(d, r, &xrow);
+  if (r < d.R) {
+    key = row_key(d, r, &xrow);
+    check_rhs_order(d, r);
+  }
   __syncthreads();
   // stable rank: rank inside the warp's equal keys + equal keys of earlier warps
   const uint32_t mask = __match_any_sync(0xFFFFFFFFu, key);
@@ -337,6 +353,7 @@ cudaError_t launch_route(const RouteArgs& a, void* ws, cudaStream_t stream) {
   d.zero_out = a.zero_out;
   d.zero_cols = a.zero_cols;
   d.zero_by_pos = a.zero_by_pos;
+  d.check_sorted = a.check_sorted;
   d.d_status = a.d_status;
   const int64_t nchunks = (R + kChunk - 1) / kChunk;
   const size_t cnt_bytes = static_cast<size_t>(32 * (a.E + 1));

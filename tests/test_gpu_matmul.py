@@ -22,19 +22,14 @@ from inputs import (bf16_bits, decode_tokens, decode_weights, dense_projections,
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["qmv", "qdec", "tc", "tc_smem", "auto"])
+@pytest.fixture(params=["qmv", "tc", "tc_smem", "auto"])
 def kernel(request, monkeypatch):
-    """Kernel choice: forced streaming (mma.sync, or tcgen05 where it supports the shape),
-    forced tensor-core tiles (weights in tensor memory where the shape allows, or staged
-    in shared memory), or the library's own plan (chosen from the most rows one expert
-    can receive)."""
-    monkeypatch.delenv("QMOE_DECODE", raising=False)
+    """Kernel choice: forced streaming, forced tensor-core tiles (weights in tensor
+    memory where the shape allows, or staged in shared memory), or the library's own
+    plan (chosen from the most rows one expert can receive)."""
     monkeypatch.delenv("QMOE_PREFILL", raising=False)
     if request.param == "auto":
         monkeypatch.delenv("QMOE_FORCE_KERNEL", raising=False)
-    elif request.param == "qdec":
-        monkeypatch.setenv("QMOE_FORCE_KERNEL", "qmv")
-        monkeypatch.setenv("QMOE_DECODE", "qdec")
     elif request.param == "tc_smem":
         monkeypatch.setenv("QMOE_FORCE_KERNEL", "tc")
         monkeypatch.setenv("QMOE_PREFILL", "tc")
@@ -100,6 +95,44 @@ def test_qmm_few_rows_equal_one_row_bitwise(gpu_lib):
         for r in range(M):
             one = host_bits16(q.qmoe_qmm(x[r:r + 1].contiguous(), *args))
             assert np.array_equal(one[0], allr[r]), (M, K, N, group, r)
+
+
+@pytest.mark.parametrize("plan", ["tmem", "smem"])
+def test_prefill_kernels_row_bits_independent_of_tile_companions(gpu_lib, monkeypatch, plan):
+    """The invariant lane of MTPLX PR #558 (Summary) asks that a row's result not depend
+    on the batch it runs in; nuvec-core quantized.rs few_row_products_equal_one_row_
+    products_bit_for_bit states it for the few-row kernels.  On the tensor-core kernels
+    (forced, weights in tensor memory or staged in shared memory) a row's output bits
+    are the same alone in its tile, among 17 or 100 rows, and in a full 192-row tile,
+    at any position; for the dense product and the SwitchGLU chain."""
+    q = gpu_lib
+    monkeypatch.setenv("QMOE_FORCE_KERNEL", "tc")
+    if plan == "smem":
+        monkeypatch.setenv("QMOE_PREFILL", "tc")
+    else:
+        monkeypatch.delenv("QMOE_PREFILL", raising=False)
+    rng = np.random.default_rng(31)
+    for bits, group, N, K in ((4, 64, 256, 2048), (8, 128, 136, 1024)):
+        w, s, b = random_qweight(rng, 1, N, K, group, bits)
+        args = (dev_u32(w[0]), dev_bf16(s[0]), dev_bf16(b[0]), group, bits)
+        X = normal_bf16(rng, (192, K))
+        full = host_bits16(q.qmoe_qmm(dev_bf16(X), *args))
+        for n in (1, 17, 100):
+            rows = rng.choice(192, size=n, replace=False)
+            sub = host_bits16(q.qmoe_qmm(dev_bf16(X[rows]), *args))
+            assert np.array_equal(sub, full[rows]), (plan, bits, n)
+    # SwitchGLU (fused up/gate + silu*mul, then down): a token's output bits with the
+    # other tokens of the call removed
+    E, H, I, T, top_k = 4, 512, 256, 160, 2
+    up, gate, down = (random_qweight(rng, E, nn, kk, 64, 4) for nn, kk in ((I, H), (I, H), (H, I)))
+    W = [qweight(*t, 64, 4) for t in (up, gate, down)]
+    x = normal_bf16(rng, (T, H))
+    idx = np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.uint32)
+    full = host_bits16(q.qmoe_switch_glu(dev_bf16(x), dev_u32(idx), *W, mode=0))
+    for n in (1, 33):
+        toks = np.sort(rng.choice(T, size=n, replace=False))
+        sub = host_bits16(q.qmoe_switch_glu(dev_bf16(x[toks]), dev_u32(idx[toks]), *W, mode=0))
+        assert np.array_equal(sub, full[toks]), (plan, "switch_glu", n)
 
 
 def test_qmm_empty(gpu_lib):
