@@ -24,10 +24,12 @@
  *   - Errors found on the device never trap: they are OR-ed into the optional
  *     `int* d_status` (device memory, caller-zeroed) as QMOE_DEV_* bits, and the
  *     rows concerned are written as zeros.
- *   - Supported codecs: group in {32, 64, 128}; bits in {1, 2, 3, 4, 5, 6, 8} for
- *     qmoe_quantize / qmoe_dequantize (the widths of nuvec-core's quantisation tests),
- *     {4, 8} and 2 (groups of 64 or 128) for the matmul calls (others return
- *     QMOE_ERR_UNSUPPORTED; 2-bit weights run on the streaming kernel); K a positive
+ *   - Supported codecs: group in {32, 64, 128}; bits in {1, 2, 3, 4, 5, 6, 8} (the widths
+ *     of nuvec-core's quantisation tests; 7 is rejected there and here) for every call.
+ *     4- and 8-bit codes run on the MMA kernels (streaming and tensor-core), 2-bit codes
+ *     in groups of 64 or 128 on the streaming MMA kernel, and 1-, 3-, 5- and 6-bit codes
+ *     and 2-bit codes in groups of 32 on a CUDA-core streaming kernel at every row count
+ *     (supported for completeness, not tuned); K a positive
  *     multiple of the group.  Packed layout: the codes of a row form one
  *     least-significant-bit-first bit stream, code j at stream bits [j*bits, (j+1)*bits)
  *     and stream bit i in bit (i mod 32) of word i/32 -- for 4 and 8 bits, code j of a

@@ -15,11 +15,10 @@ bool group_ok(int group) { return group == 32 || group == 64 || group == 128; }
 bool codec_ok(int group, int bits) {
   return (bits >= 1 && bits <= 8 && bits != 7) && group_ok(group);
 }
-// the matmul kernels: 4- and 8-bit codes, and 2-bit codes in groups of 64 or 128
-bool matmul_codec_ok(int group, int bits) {
-  if (bits == 2) return group == 64 || group == 128;
-  return (bits == 4 || bits == 8) && group_ok(group);
-}
+// the matmul calls: every codec width (4- and 8-bit codes, and 2-bit codes in groups of
+// 64 or 128, on the MMA kernels; 1-, 3-, 5- and 6-bit codes and 2-bit codes in groups of
+// 32 on the bit-stream kernel)
+bool matmul_codec_ok(int group, int bits) { return codec_ok(group, bits); }
 
 // K must be a positive multiple of the group size.
 int check_codec(int64_t K, int group, int bits) {
@@ -196,13 +195,18 @@ int qmoe_qmm(const qmoe_bf16* x, int64_t M, const uint32_t* codes, const qmoe_bf
   a.dense_rows = M;
   a.d_status = d_status;
   // one weight matrix: tensor cores from 32 rows, else the streaming kernel
+  auto s = static_cast<cudaStream_t>(stream);
+  if (qmv_bits_needed(bits, group)) {  // bit-stream widths: one kernel at every row count
+    a.bm = M > 8 ? 16 : 8;
+    a.max_tiles = (M + a.bm - 1) / a.bm;
+    return cuda_status(launch_qmv_bits(a, s));
+  }
   const Kernel k = forced_kernel();
   const bool big = k == Kernel::Tc || (k == Kernel::Auto && M >= 32);
   const bool ts = big && ts_allowed() && qmm_ts_supported(a);
   const bool tc = !ts && big && qmm_tc_supported(a);
   a.bm = ts ? kTsTileRows : tc ? kTcBm : (M > 8 ? 16 : 8);
   a.max_tiles = (M + a.bm - 1) / a.bm;
-  auto s = static_cast<cudaStream_t>(stream);
   if (ts) return cuda_status(launch_qmm_ts(a, s));
   return cuda_status(tc ? launch_qmm_tc(a, s) : launch_qmv(a, s));
 }
@@ -289,9 +293,9 @@ int qmoe_gather_qmm(const qmoe_bf16* x, int64_t x_batches, int64_t M, int64_t K,
     a.src_row = nullptr;
     return cuda_status(pl.ts ? launch_qmm_ts(a, s) : launch_qmm_tc(a, s));
   }
-  a.x = x;  // the streaming kernel reads x through src_row
+  a.x = x;  // the streaming kernels read x through src_row
   a.src_row = rb.src_row;
-  return cuda_status(launch_qmv(a, s));
+  return cuda_status(qmv_bits_needed(bits, group) ? launch_qmv_bits(a, s) : launch_qmv(a, s));
 }
 
 size_t qmoe_gather_mm_workspace_size(int64_t B, int64_t M, int64_t E, int64_t N, int64_t K) {
@@ -467,8 +471,11 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   // picks the plan: any routing is served correctly by either kernel.
   GemmArgs ug_sorted = ug;  // as the tensor-core streaming kernel would read x
   ug_sorted.src_row = nullptr;
-  const Plan pl = plan_for(R, E, T, qmm_tc_supported(ug) && qmm_tc_supported(dn),
-                           qmm_ts_supported(ug_sorted) && qmm_ts_supported(dn));
+  const bool bits_ug = qmv_bits_needed(ug.bits, ug.group);
+  const bool bits_dn = qmv_bits_needed(dn.bits, dn.group);
+  const bool mma_only = !bits_ug && !bits_dn;  // tensor-core plans take no bit-stream width
+  const Plan pl = plan_for(R, E, T, mma_only && qmm_tc_supported(ug) && qmm_tc_supported(dn),
+                           mma_only && qmm_ts_supported(ug_sorted) && qmm_ts_supported(dn));
   ug.bm = dn.bm = pl.bm;
   ug.max_tiles = dn.max_tiles = max_tiles_for(R, E, pl.bm);
 
@@ -505,8 +512,8 @@ int qmoe_switch_glu(const qmoe_bf16* x, const uint32_t* indices, int64_t T, int 
   }
   ug.x = x;
   ug.src_row = rb.src_row;
-  if (launch_qmv(ug, s) != cudaSuccess) return QMOE_ERR_CUDA;
-  return cuda_status(launch_qmv(dn, s));
+  if ((bits_ug ? launch_qmv_bits(ug, s) : launch_qmv(ug, s)) != cudaSuccess) return QMOE_ERR_CUDA;
+  return cuda_status(bits_dn ? launch_qmv_bits(dn, s) : launch_qmv(dn, s));
 }
 
 int qmoe_moe_combine(const qmoe_bf16* y_sorted, const uint32_t* inv_order, const float* scores,

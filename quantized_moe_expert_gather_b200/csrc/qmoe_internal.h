@@ -130,6 +130,10 @@ struct GemmArgs {
 // launch's last CTA leaves unissued, or -1.  Read and cleared by that launch.
 int64_t take_skip_stage();
 cudaError_t launch_qmv(const GemmArgs& a, cudaStream_t stream);   // tiles of <= 16 rows
+// Bit-stream code widths (1, 3, 5, 6 bits; 2 bits in groups of 32): CUDA-core streaming
+// kernel over tiles of <= 16 rows.  qmv_bits_needed: the codec has no MMA kernel.
+bool qmv_bits_needed(int bits, int group);
+cudaError_t launch_qmv_bits(const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_qmm_tc(const GemmArgs& a, cudaStream_t stream); // tiles of 128 rows
 bool qmm_tc_supported(const GemmArgs& a);
 // Tensor-core kernel with the dequantised weights as the MMA A operand in tensor memory,

@@ -68,17 +68,18 @@ def test_matmuls_reject_bad_arguments_on_host(lib):
     assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 63, 64, 4, fake, None, None) == ERR_ARG
     # unsupported codec
     assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 96, 48, 4, fake, None, None) == ERR_UNSUPPORTED
-    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 96, 32, 3, fake, None, None) == ERR_UNSUPPORTED
-    # 2-bit matmuls need groups of 64 or 128; 1-bit codes have no matmul kernel
-    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 64, 32, 2, fake, None, None) == ERR_UNSUPPORTED
-    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 64, 64, 1, fake, None, None) == ERR_UNSUPPORTED
+    # every width of the quantisation tests has a matmul; 7 bits (rejected there), 0 and
+    # 9 bits do not
+    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 96, 32, 7, fake, None, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 64, 32, 0, fake, None, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_qmm(fake, 3, fake, fake, fake, 8, 64, 64, 9, fake, None, None) == ERR_UNSUPPORTED
     assert lib.qmoe_qmm(fake, 0, fake, fake, fake, 8, 64, 64, 4, fake, None, None) == 0
     # gather: workspace too small
     need = lib.qmoe_gather_qmm_workspace_size(4, 1, 8, 16, 64)
     assert need > 0
     assert lib.qmoe_gather_qmm(fake, 4, 1, 64, fake, fake, fake, 8, 16, 64, 4, None, fake, 4, 0,
                                fake, need - 1, fake, None, None) == ERR_WORKSPACE
-    assert lib.qmoe_gather_qmm(fake, 4, 1, 64, fake, fake, fake, 8, 16, 64, 5, None, fake, 4, 0,
+    assert lib.qmoe_gather_qmm(fake, 4, 1, 64, fake, fake, fake, 8, 16, 64, 7, None, fake, 4, 0,
                                fake, need, fake, None, None) == ERR_UNSUPPORTED
     # combine: hidden size not a multiple of 8, and a gate without a shared expert
     assert lib.qmoe_moe_combine(fake, fake, fake, fake, None, None, 2, 2, 12, fake, None, None) == ERR_UNSUPPORTED

@@ -135,6 +135,65 @@ def test_prefill_kernels_row_bits_independent_of_tile_companions(gpu_lib, monkey
         assert np.array_equal(sub, full[toks]), (plan, "switch_glu", n)
 
 
+# bit-stream widths (1, 3, 5, 6 bits; 2 bits in groups of 32): the CUDA-core kernel
+BITSTREAM_QMM = [  # (M, N, K, bits, group)
+    (1, 64, 512, 3, 64), (5, 33, 256, 5, 32), (17, 40, 384, 6, 128), (3, 64, 256, 1, 64),
+    (4, 48, 320, 2, 32), (40, 37, 512, 3, 32), (2, 16, 1024, 6, 64), (9, 24, 128, 5, 128),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bits,group", BITSTREAM_QMM)
+def test_qmm_bitstream_widths(gpu_lib, M, N, K, bits, group):
+    """quantized_matmul over the widths of nuvec-core quantized.rs `const BITS` whose codes
+    straddle words (3, 5, 6) or have no MMA kernel here (1; 2 in groups of 32): ragged N,
+    several 16-row tiles."""
+    q = gpu_lib
+    rng = np.random.default_rng(M * 11 + N + K + bits)
+    w, s, b = random_qweight(rng, 1, N, K, group, bits)
+    x = normal_bf16(rng, (M, K))
+    want = O.qmm(x, w[0], s[0], b[0], group, bits)
+    y = q.qmoe_qmm(dev_bf16(x), dev_u32(w[0]), dev_bf16(s[0]), dev_bf16(b[0]), group, bits)
+    assert_close(f"qmm {M}x{N}x{K} {bits}-bit g{group}", y, want)
+
+
+@pytest.mark.parametrize("bits,group", [(1, 32), (2, 32), (3, 64), (5, 128), (6, 32)])
+def test_gather_qmm_bitstream_widths(gpu_lib, bits, group):
+    """gather_qmm over the bit-stream widths: sorted and unsorted indices give the same
+    bits; rows of one x batch broadcast over its experts."""
+    q = gpu_lib
+    rng = np.random.default_rng(bits * 7 + group)
+    E, N, K = 8, 48, 256
+    w, s, b = random_qweight(rng, E, N, K, group, bits)
+    x = normal_bf16(rng, (12, 1, K))
+    rhs = np.stack([rng.choice(E, size=3, replace=False) for _ in range(12)]).reshape(-1)
+    rhs = rhs.astype(np.uint32)
+    W = (dev_u32(w), dev_bf16(s), dev_bf16(b))
+    want = O.gather_qmm(x, w, s, b, group, bits, None, rhs)
+    y = q.qmoe_gather_qmm(dev_bf16(x), *W, None, dev_u32(rhs), group, bits)
+    assert_close(f"gather {bits}-bit g{group}", y, want)
+    perm = np.argsort(rhs, kind="stable")
+    lhs = (np.arange(rhs.size) // 3)[perm].astype(np.uint32)
+    ys = q.qmoe_gather_qmm(dev_bf16(x), *W, dev_u32(lhs), dev_u32(rhs[perm]), group, bits,
+                           sorted_indices=True)
+    assert np.array_equal(host_bits16(ys), host_bits16(y)[perm])
+
+
+@pytest.mark.parametrize("T,bits,group", [(4, 3, 64), (64, 5, 32), (24, 6, 128), (8, 1, 64)])
+def test_switch_glu_bitstream_widths(gpu_lib, T, bits, group):
+    """SwitchGLU with bit-stream codes (fused up/gate + silu*mul, then down), decode- and
+    prefill-sized rows per expert."""
+    q = gpu_lib
+    rng = np.random.default_rng(T + bits + group)
+    E, H, I, top_k = 8, 512, 256, 2
+    up, gate, down = (random_qweight(rng, E, n, k, group, bits) for n, k in ((I, H), (I, H), (H, I)))
+    x = normal_bf16(rng, (T, H))
+    idx = np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.uint32)
+    W = [qweight(*t, group, bits) for t in (up, gate, down)]
+    y = q.qmoe_switch_glu(dev_bf16(x), dev_u32(idx), *W, mode=0)
+    want, _ = O.switch_glu(x, idx, (*up, group, bits), (*gate, group, bits), (*down, group, bits))
+    assert_close(f"switch_glu {bits}-bit g{group} T={T}", y, want)
+
+
 def test_qmm_empty(gpu_lib):
     q = gpu_lib
     x = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")

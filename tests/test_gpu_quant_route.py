@@ -9,8 +9,8 @@ import pytest
 import torch
 
 import oracle as O
-from gpu_util import dev_u32, host_bits16, host_u32
-from inputs import bf16_bits
+from gpu_util import assert_close, dev_bf16, dev_u32, host_bits16, host_u32
+from inputs import bf16_bits, normal_bf16
 
 pytestmark = pytest.mark.gpu
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
@@ -55,18 +55,24 @@ def test_quantize_dequantize_bit_exact(gpu_lib, bits, group, dtype):
     assert np.array_equal(host_bits16(d16), O.bf16_from_f32(want_d))
 
 
-def test_codec_widths_outside_the_kernels_are_rejected(gpu_lib):
-    """7 bits is rejected by the codec ([P3] rejected_arguments); widths other than 4
-    and 8 quantise and dequantise but are rejected by the matmul calls."""
+def test_seven_bits_rejected_and_quantised_3bit_weights_multiply(gpu_lib):
+    """7 bits is rejected by the codec and the matmuls ([P3] rejected_arguments); 3-bit
+    weights quantised on the GPU go straight into qmoe_qmm (the bit-stream layout is the
+    matmul's input layout) and match the oracle's product of the same codes."""
     q = gpu_lib
     w = torch.zeros((2, 64), dtype=torch.float32, device="cuda")
     with pytest.raises(RuntimeError, match="UNSUPPORTED"):
         q.qmoe_quantize(w, 64, 7)
-    codes, s, b = q.qmoe_quantize(w.to(torch.bfloat16), 64, 3)
-    assert codes.shape == (2, 6)
-    x = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")
+    rng = np.random.default_rng(3)
+    wb = torch.from_numpy(rng.standard_normal((40, 192)).astype(np.float32)).cuda().to(torch.bfloat16)
+    codes, s, b = q.qmoe_quantize(wb, 64, 3)
+    assert codes.shape == (40, 18)
+    xh = normal_bf16(rng, (3, 192))
+    y = q.qmoe_qmm(dev_bf16(xh), codes, s, b, 64, 3)
+    want = O.qmm(xh, host_u32(codes), host_bits16(s), host_bits16(b), 64, 3)
+    assert_close("3-bit qmm of GPU-quantised weights", y, want)
     with pytest.raises(RuntimeError, match="UNSUPPORTED"):
-        q.qmoe_qmm(x, codes, s, b, 64, 3)
+        q.qmoe_qmm(dev_bf16(xh), codes, s, b, 64, 7)
 
 
 @pytest.mark.parametrize("R,E", [(1, 1), (37, 5), (1024, 288), (1025, 256), (4099, 8),
