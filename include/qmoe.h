@@ -247,6 +247,26 @@ QMOE_API int qmoe_sort_by_expert(const uint32_t* indices, int64_t R, int64_t E, 
                         size_t workspace_bytes, int* d_status, qmoe_stream stream);
 
 /*
+ * qmoe_ep_pack -- the send buffer of an expert-parallel dispatch ([P5] Change: the sorted
+ * chain gathers routed rows in expert order and keeps the inverse permutation for the
+ * combine).  With experts partitioned contiguously over ranks (expert e on rank
+ * e / E_local), rows in expert order are grouped by owner rank: one all-to-all of these
+ * buffers dispatches every row, the same all-to-all in reverse returns the outputs in
+ * expert order for qmoe_moe_combine (with the sort's inv_order).
+ *   x        [T, H] bf16 activations;  indices [T, top_k] uint32 expert ids
+ *   order    [T*top_k] uint32 from qmoe_sort_by_expert(indices)
+ *   x_send   [T*top_k, H] bf16 (out): x_send[p] = x[order[p] / top_k]
+ *   e_send   [T*top_k] uint32 (out): indices[order[p]] mod E_local, the expert's number
+ *            on its owner rank
+ * H must be a multiple of 8 (QMOE_ERR_UNSUPPORTED); x and x_send 16-byte aligned.
+ * Rows past the valid ones (index >= E) are packed too; a caller sends only the first
+ * offsets[E] rows.  QMOE_ERR_ARG for bad sizes or pointers.
+ */
+QMOE_API int qmoe_ep_pack(const qmoe_bf16* x, int64_t T, int64_t H, int top_k,
+                          const uint32_t* indices, const uint32_t* order, int64_t E_local,
+                          qmoe_bf16* x_send, uint32_t* e_send, int* d_status, qmoe_stream stream);
+
+/*
  * qmoe_tile_table -- expert-aligned row tiles ([P2] Proposed changes: every tile gets
  * the row to start from, the expert to load and the number of valid rows; no tile
  * spans two experts).

@@ -22,6 +22,7 @@ __all__ = [
     "QmoeError", "load", "library_path", "qmoe_status_string", "qmoe_launch_count", "qmoe_timing_enable", "qmoe_timing_read",
     "qmoe_quantize", "qmoe_dequantize", "qmoe_qmm", "qmoe_gather_qmm",
     "qmoe_gather_qmm_workspace_size", "qmoe_gather_qmm_noalloc", "qmoe_sort_by_expert", "qmoe_tile_table",
+    "qmoe_ep_pack",
     "qmoe_switch_glu", "qmoe_switch_glu_workspace_size", "qmoe_moe_combine",
     "qmoe_moe_combine_stock", "qmoe_gather_mm", "qmoe_gather_mm_workspace_size", "QWeight",
     "QMOE_DEV_BAD_INDEX", "QMOE_DEV_TIMEOUT", "QMOE_DEV_UNSORTED", "qmoe_debug_skip_stage",
@@ -64,6 +65,7 @@ _SIGS = {
     "qmoe_sort_by_expert_workspace_size": (_sz, [_i64, _i64]),
     "qmoe_sort_by_expert": (_i32, [_p, _i64, _i64, _p, _p, _p, _p, _sz, _p, _p]),
     "qmoe_tile_table": (_i32, [_p, _i64, _i32, _p, _i64, _p, _p, _p]),
+    "qmoe_ep_pack": (_i32, [_p, _i64, _i64, _i32, _p, _p, _i64, _p, _p, _p, _p]),
     "qmoe_switch_glu_workspace_size": (_sz, [_i64, _i32, ctypes.POINTER(_QWeight),
                                              ctypes.POINTER(_QWeight), ctypes.POINTER(_QWeight)]),
     "qmoe_switch_glu": (_i32, [_p, _p, _i64, _i32, ctypes.POINTER(_QWeight),
@@ -295,6 +297,28 @@ def qmoe_sort_by_expert(indices, E: int, status=None):
         _ptr(indices), R, E, _ptr(order), _ptr(inv), _ptr(offsets), _ptr(ws), need, _ptr(status),
         _stream()))
     return order, inv, offsets
+
+
+def qmoe_ep_pack(x, indices, order, E_local: int, x_send=None, e_send=None, status=None):
+    """Expert-parallel send buffers: ``x_send[p] = x[order[p] // top_k]`` and
+    ``e_send[p] = indices.flat[order[p]] % E_local`` for the rows in expert order.
+    Returns ``(x_send [T*top_k, H] bf16, e_send [T*top_k] int32)``."""
+    _need(x, "x", _BF16)
+    _need(indices, "indices", _IDX)
+    _need(order, "order", _IDX)
+    T, H = x.shape
+    top_k = indices.shape[1]
+    R = T * top_k
+    if order.numel() != R:
+        raise ValueError("order must hold T*top_k entries")
+    if x_send is None:
+        x_send = torch.empty((R, H), dtype=torch.bfloat16, device=x.device)
+    if e_send is None:
+        e_send = torch.empty(R, dtype=torch.int32, device=x.device)
+    _check("qmoe_ep_pack", load().qmoe_ep_pack(
+        _ptr(x), T, H, top_k, _ptr(indices), _ptr(order), E_local, _ptr(x_send), _ptr(e_send),
+        _ptr(status), _stream()))
+    return x_send, e_send
 
 
 def qmoe_tile_table(offsets, bm: int, max_tiles: int, status=None):
