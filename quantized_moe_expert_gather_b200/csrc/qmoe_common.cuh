@@ -84,19 +84,23 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
+// One test of the phase; the thread may be suspended until the phase completes or for up
+// to kWaitHintNs, so a waiting warp does not keep issuing while it waits.
+constexpr uint32_t kWaitHintNs = 1000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
       : "memory");
   return ok != 0;
 }
 
-// Spin limit for every mbarrier wait: about a second with the back-off below.
+// Spin limit for every mbarrier wait: about a second with the back-off below (up to a few
+// seconds when every test is suspended for its full hint).
 constexpr uint32_t kWaitSpins = 1u << 22;
 
 // Waits until the phase of `bar` with parity `parity` has completed.  Returns

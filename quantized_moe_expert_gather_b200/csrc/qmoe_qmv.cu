@@ -391,39 +391,34 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
   auto chunk_groups = [&](int64_t ch) -> int {
     return static_cast<int>(imin64(C::KB_PER_CHUNK, KB_TOTAL - ch * C::KB_PER_CHUNK));
   };
-  // This lane's activation pointers for unit u (null for empty token slots).
+  // This lane's activation pointers for unit u.  A token slot past the tile's valid rows
+  // reads the tile's first row: its MMA column is never stored, so any finite values
+  // serve, and the loads need no branch.
   auto tile_rows = [&](int64_t u, TileInfo& ti, const uint16_t* (&rows)[NT]) {
     ti = tile_info<NT>(p, u / NB);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint32_t slot = g + 8 * nt;
-      rows[nt] = nullptr;
-      if (slot < ti.valid) {
-        const uint32_t pos = ti.row_start + slot;
-        const uint32_t sr = p.src_row ? p.src_row[pos] : pos;
-        rows[nt] = p.x + static_cast<int64_t>(sr) * p.K + x_off;
-      }
+      const uint32_t pos = ti.row_start + (slot < ti.valid ? slot : 0u);
+      const uint32_t sr = p.src_row ? p.src_row[pos] : pos;
+      rows[nt] = p.x + static_cast<int64_t>(sr) * p.K;
     }
   };
-  // Issues the loads of chunk `ch` for the given rows into `dst`.
+  // Issues the loads of chunk `ch` for the given rows into `dst`; a group past the chunk's
+  // last one (never computed) reads the row's first activations, always in bounds.
   auto load_x = [&](const uint16_t* const (&rows)[NT], int64_t ch, XBuf& dst) {
     const int nkb = chunk_groups(ch);
 #pragma unroll
     for (int i = 0; i < C::KB_PER_WARP; ++i) {
-      const bool live = warp + C::CW * i < nkb;
+      const int64_t off = warp + C::CW * i < nkb ? ch * CHUNK_ELEMS + x_off + i * C::CW * GS : 0;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int j = 0; j < C::WORDS * C::XW; ++j) {
-          if constexpr (BITS != 8) {  // 8 activations per vector, XW vectors per code word
-            dst[i][nt][j] = make_uint4(0, 0, 0, 0);
-            if (rows[nt] != nullptr && live)
-              dst[i][nt][j] = ldg_nc_v4(rows[nt] + ch * CHUNK_ELEMS + i * C::CW * GS + 8 * j);
-          } else {
-            dst[i][nt][j] = make_uint2(0, 0);
-            if (rows[nt] != nullptr && live)
-              dst[i][nt][j] = ldg_nc_v2(rows[nt] + ch * CHUNK_ELEMS + i * C::CW * GS + 4 * j);
-          }
+          if constexpr (BITS != 8)  // 8 activations per vector, XW vectors per code word
+            dst[i][nt][j] = ldg_nc_v4(rows[nt] + off + 8 * j);
+          else
+            dst[i][nt][j] = ldg_nc_v2(rows[nt] + off + 4 * j);
         }
     }
   };
