@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
           if constexpr (C::WBF16) {
             // bf16 weight tiles, 128 rows x 64 k per stack, straight into the weight ring
             const uint32_t s2 = it % kS2;
-            if (!mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+            if (!mbar_wait<false>(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
             mbar_arrive_expect_tx(&full2[s2], C::B_BYTES);
 #pragma unroll
             for (int m = 0; m < 2; ++m)
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
           } else {
             if (sb_first(ks)) {
               const uint32_t e = sbit & 1;
-              if (!mbar_wait(&empty_sb[e], ((sbit >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+              if (!mbar_wait<false>(&empty_sb[e], ((sbit >> 1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
               if constexpr (SB_WHOLE) {
                 // rows wrow.. of one stack are contiguous: [128 rows][sb_groups] per array
                 const uint32_t bytes = kBM * p.sb_groups * 2;
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
             if (ks % C::PK == 0) {
               // packed codes of the next PK stages: 128 bytes of each row, 128B-swizzled
               const uint32_t ps = pbit % C::SP;
-              if (!mbar_wait(&emptyP[ps], ((pbit / C::SP) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+              if (!mbar_wait<false>(&emptyP[ps], ((pbit / C::SP) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
               mbar_arrive_expect_tx(&fullP[ps], C::P_SLOT);
   #pragma unroll
               for (int m = 0; m < 2; ++m)
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
             }
           }
           const uint32_t s1 = it % kS1;
-          if (!mbar_wait(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
+          if (!mbar_wait<false>(&empty1[s1], ((it / kS1) & 1) ^ 1, p.d_status)) { *abort_flag = 1; ab = true; break; }
           mbar_arrive_expect_tx(&full1[s1], C::A_BYTES);
           tma_load_2d(smem + C::OFF_A + s1 * C::A_BYTES, &p.tm_a, &full1[s1],
                       static_cast<int32_t>(ks * kBK), static_cast<int32_t>(tl.row_start));
@@ -289,16 +289,16 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
       if (ab) {
         // let the copies already issued land before the CTA can exit
         const uint32_t first = it > static_cast<uint32_t>(kS1) ? it - kS1 : 0u;
-        for (uint32_t k = first; k < it; ++k) mbar_wait(&full1[k % kS1], (k / kS1) & 1, nullptr);
+        for (uint32_t k = first; k < it; ++k) mbar_wait<false>(&full1[k % kS1], (k / kS1) & 1, nullptr);
         const uint32_t sfirst = sbit > 2u ? sbit - 2 : 0u;
-        for (uint32_t k = sfirst; k < sbit; ++k) mbar_wait(&full_sb[k & 1], (k >> 1) & 1, nullptr);
+        for (uint32_t k = sfirst; k < sbit; ++k) mbar_wait<false>(&full_sb[k & 1], (k >> 1) & 1, nullptr);
         if constexpr (C::WBF16) {
           const uint32_t bfirst = it > static_cast<uint32_t>(kS2) ? it - kS2 : 0u;
-          for (uint32_t k = bfirst; k < it; ++k) mbar_wait(&full2[k % kS2], (k / kS2) & 1, nullptr);
+          for (uint32_t k = bfirst; k < it; ++k) mbar_wait<false>(&full2[k % kS2], (k / kS2) & 1, nullptr);
         } else {
           const uint32_t pfirst = pbit > static_cast<uint32_t>(C::SP) ? pbit - C::SP : 0u;
           for (uint32_t k = pfirst; k < pbit; ++k)
-            mbar_wait(&fullP[k % C::SP], (k / C::SP) & 1, nullptr);
+            mbar_wait<false>(&fullP[k % C::SP], (k / C::SP) & 1, nullptr);
         }
       }
     }
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     int ok = 1;
     for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
       const uint32_t buf = tc & 1;
-      if (lane == 0) ok = !*abort_flag && mbar_wait(&tempty[buf], ((tc >> 1) & 1) ^ 1, p.d_status);
+      if (lane == 0) ok = !*abort_flag && mbar_wait<false>(&tempty[buf], ((tc >> 1) & 1) ^ 1, p.d_status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         if (lane == 0) *abort_flag = 1;
         break;
@@ -322,8 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
       for (int64_t ks = 0; ks < KS; ++ks, ++it) {
         const uint32_t s1 = it % kS1, s2 = it % kS2;
         if (lane == 0)
-          ok = mbar_wait(&full1[s1], (it / kS1) & 1, p.d_status) &&
-               mbar_wait(&full2[s2], (it / kS2) & 1, p.d_status);
+          ok = mbar_wait<false>(&full1[s1], (it / kS1) & 1, p.d_status) &&
+               mbar_wait<false>(&full2[s2], (it / kS2) & 1, p.d_status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
           if (lane == 0) *abort_flag = 1;
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     const bool leader = elect_one();
     if (leader && issued && *abort_flag) {
       tc_commit(drain);  // completes when every MMA issued so far has finished
-      mbar_wait(drain, 0, nullptr);
+      mbar_wait<false>(drain, 0, nullptr);
     }
     __syncwarp();
   } else if (warp >= kDqWarp0) {
@@ -367,11 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
           if (*abort_flag) break;
           const uint32_t e = sbit & 1;
           if (sb_first(ks) &&
-              !mbar_wait(&full_sb[e], (sbit >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
+              !mbar_wait<false>(&full_sb[e], (sbit >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
           const uint32_t ps = pbit % C::SP, s2 = it % kS2;
           if (ks % C::PK == 0 &&
-              !mbar_wait(&fullP[ps], (pbit / C::SP) & 1, p.d_status)) { *abort_flag = 1; break; }
-          if (!mbar_wait(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
+              !mbar_wait<false>(&fullP[ps], (pbit / C::SP) & 1, p.d_status)) { *abort_flag = 1; break; }
+          if (!mbar_wait<false>(&empty2[s2], ((it / kS2) & 1) ^ 1, p.d_status)) { *abort_flag = 1; break; }
           const int pj = static_cast<int>(ks % C::PK);  // stage inside the packed rows
           const int gin = sb_whole ? static_cast<int>(ks * kBK / GS)
                                    : static_cast<int>((ks * kBK / GS) % kSbGroups);
@@ -434,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_tc_kernel(const __grid_consta
     for (int64_t u = u_begin; u < u_end; u += u_step, ++tc) {
       if (*abort_flag) break;
       const uint32_t buf = tc & 1;
-      if (!mbar_wait(&tfull[buf], (tc >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
+      if (!mbar_wait<false>(&tfull[buf], (tc >> 1) & 1, p.d_status)) { *abort_flag = 1; break; }
       tc_fence_after();
       const Tile tl = tc_tile(p, u / NBLK);
       const int64_t n0 = (u % NBLK) * unit_n;
