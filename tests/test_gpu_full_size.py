@@ -12,6 +12,8 @@
   4-bit group 64 and 8-bit group 128 (MTPLX PR #558, Tests: the row counts of its block
   checks): the routed rows as above, and the block output on 160 sampled tokens, whose
   oracle chain feeds its own bf16 expert and shared outputs to its combine.
+* Unquantized gather_mm on the benchmarked workload (2048 -> 512, 256 experts, Zipf top-8)
+  at T = 4096 and 16384 tokens, on sampled routed rows.
 
 Tolerance as everywhere: |got - want| <= 8e-3 * max|want| over the compared values.
 """
@@ -143,3 +145,43 @@ def test_moe_block_full_size(gpu_lib, monkeypatch, T, bits, group):
                          d["w_sg"])
     assert_close(f"block T={T} {bits}-bit g{group} output of {toks.size} tokens",
                  out[torch.from_numpy(toks).cuda()], want)
+
+
+_GMM = {}
+
+
+def _gather_mm_case(T):
+    """The bench's gather_mm workload (the weights, then the activations of T = 4096 and of
+    T = 16384 from the same seeded stream), the sampled routed rows of T tokens and the
+    oracle's values there (over the sampled rows' experts only)."""
+    from inputs import normal_bf16, prefill_routing
+    E, K, N = 256, 2048, 512
+    if "w" not in _GMM:
+        rng = np.random.default_rng(21)
+        _GMM["w"] = normal_bf16(rng, (E, N, K), 1 / np.sqrt(K))
+        _GMM["x"] = {t: normal_bf16(rng, (t, 1, K)) for t in (4096, 16384)}
+    if _GMM.get("T") != T:
+        w, x = _GMM["w"], _GMM["x"][T]
+        idx, _ = prefill_routing(0, T, E, TOP_K)
+        rhs = idx.reshape(-1).astype(np.uint32)
+        order, _, offsets = O.sort_by_expert(rhs, E)
+        b = np.sort(order[sample_positions(offsets, seed=T)].astype(np.int64))
+        ue = np.unique(rhs[b])
+        want = O.gather_mm(x[b // TOP_K], w[ue], np.arange(b.size), np.searchsorted(ue, rhs[b]))
+        _GMM.update(T=T, case=(x, w, rhs, b, want))
+    return _GMM["case"]
+
+
+@pytest.mark.parametrize("T", [4096, 16384])
+def test_gather_mm_full_size(gpu_lib, monkeypatch, T):
+    """Unquantized gather_mm on the benchmarked workload (hidden 2048 -> 512, 256 experts,
+    Zipf-skewed top-8 routing of T tokens, x broadcast over each token's experts; MLX PR
+    #4567, Description: the gather_mm whose row tiles the page reorganises), compared with
+    the oracle on sampled routed rows chosen as for the prefill layer."""
+    q = gpu_lib
+    _set_plan(monkeypatch, "auto")
+    x, w, rhs, b, want = _gather_mm_case(T)
+    got = q.qmoe_gather_mm(dev_bf16(x), dev_bf16(w), None, dev_u32(rhs))
+    torch.cuda.synchronize()
+    assert_close(f"gather_mm T={T}: {b.size} sampled rows",
+                 got[torch.from_numpy(b).cuda()], want)

@@ -394,6 +394,8 @@ GATHER_MM_CASES = [  # (x_batches, M, K, E, N, B)
     (300, 1, 512, 8, 200, 300),   # rows across three 128-row tiles; N not a multiple of 128
     (40, 1, 256, 5, 384, 320),    # x broadcast over 8 experts per token
     (3, 7, 128, 4, 64, 3),        # several rows per batch, one tile
+    (1000, 1, 256, 3, 136, 1000), # several 128-row tiles per expert with ragged tails
+    (50, 2, 192, 6, 128, 50),     # K of three 64-k stages
 ]
 
 
