@@ -72,10 +72,11 @@ struct Cfg {
   static constexpr int THREADS = (CW + 2) * 32;  // consumers, producer, epilogue
   static constexpr int KB_BYTES = GS * BITS / 8;                 // one group of one row
   // 1 KB of each row per stage (512 B with two token sets, whose doubled register
-  // arrays would otherwise spill; half that for 2-bit codes, whose activations per
-  // code byte are twice as many), at least one group per consumer warp
+  // arrays would otherwise spill, and with four 16-row blocks, whose stage it keeps at
+  // 32 KB; half that for 2-bit codes, whose activations per code byte are twice as many),
+  // at least one group per consumer warp
   static constexpr int CHUNK_ROW_BYTES =
-      std::max((NT == 2 ? 512 : 1024) / (BITS == 2 ? 2 : 1), KB_BYTES * CW);
+      std::max((NT == 2 || NMAT == 4 ? 512 : 1024) / (BITS == 2 ? 2 : 1), KB_BYTES * CW);
   static constexpr int KB_PER_CHUNK = CHUNK_ROW_BYTES / KB_BYTES;
   static constexpr int KB_PER_WARP = KB_PER_CHUNK / CW;
   static constexpr int BOXES = CHUNK_ROW_BYTES / 128;
@@ -117,7 +118,7 @@ struct alignas(64) QmvParams {
   const uint32_t* num_tiles;
   int64_t dense_rows;
   int64_t N, K, E;
-  int pair;                     // 1: one weight stack, a unit is two adjacent 16-row blocks
+  int pair;                     // 1: one weight stack, a unit is NMAT adjacent 16-row blocks
   int code3d;                   // codes by one 3-D box per 16-row block (else one 2-D box per 128 B)
   int sb_tma;                   // scales/biases by TMA (row pitch a multiple of 16 bytes)
   int sb_vec;                   // else: byte width of the copy pieces (2: plain copies)
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 
   const int64_t KB_TOTAL = p.K / GS;
   const int64_t NCH = (KB_TOTAL + C::KB_PER_CHUNK - 1) / C::KB_PER_CHUNK;
-  const int unit_rows = p.pair ? 2 * kRows : kRows;  // output channels per unit
+  const int unit_rows = p.pair ? NMAT * kRows : kRows;  // output channels per unit
   const int64_t NB = (p.N + unit_rows - 1) / unit_rows;
   const int64_t units = num_tiles<NT>(p) * NB;
   const int64_t u_begin = units * blockIdx.x / gridDim.x;
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
     // ------------------------------------------------------------- producer
     if (lane == 0) {
 #pragma unroll
-      for (int m = 0; m < NMAT; ++m) {
+      for (int m = 0; m < 2; ++m) {
         tma_prefetch_desc(&p.tmap[m]);
         if (p.sb_tma) {
           tma_prefetch_desc(&p.tmap_sb[m][0]);
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
           if (p.code3d) {
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
-              tma_load_3d(st + m * C::BOXES * 2048, &p.tmap[m], &full[stage], 0,
+              tma_load_3d(st + m * C::BOXES * 2048, &p.tmap[p.pair ? 0 : m], &full[stage], 0,
                           static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)),
                           static_cast<int32_t>(ch * C::BOXES));
           } else {
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
               for (int bx = 0; bx < C::BOXES; ++bx)
-                tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[m], &full[stage],
+                tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[p.pair ? 0 : m], &full[stage],
                             xw + bx * 32, static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
           }
           if (p.sb_tma) {
@@ -265,7 +266,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 #pragma unroll
               for (int arr = 0; arr < 2; ++arr)
                 tma_load_2d(st + C::CODE_BYTES + (m * 2 + arr) * kRows * C::KB_PER_CHUNK * 2,
-                            &p.tmap_sb[m][arr], &full[stage], xg,
+                            &p.tmap_sb[p.pair ? 0 : m][arr], &full[stage], xg,
                             static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
           }
         }
@@ -284,8 +285,9 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
           const int arr = (tk / (pieces * kRows)) % 2;
           const int m = tk / (pieces * kRows * 2);
           const int mrow = p.pair ? kRows * m + rr : rr;  // row inside the unit
-          if (mrow >= (p.pair ? static_cast<int>(imin64(2 * kRows, p.N - n0)) : nrows)) continue;
-          const uint16_t* src = (arr ? p.biases[m] : p.scales[m]) + (row0 + mrow) * KB_TOTAL + kb0;
+          if (mrow >= (p.pair ? static_cast<int>(imin64(NMAT * kRows, p.N - n0)) : nrows)) continue;
+          const int sm = p.pair ? 0 : m;  // the weight stack
+          const uint16_t* src = (arr ? p.biases[sm] : p.scales[sm]) + (row0 + mrow) * KB_TOTAL + kb0;
           uint16_t* dst = sb + ((m * 2 + arr) * kRows + rr) * C::KB_PER_CHUNK;
           const int off = piece * (p.sb_vec / 2);
           if (p.sb_vec == 16)
@@ -704,7 +706,17 @@ cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
 
 template <int BITS, int GS>
 cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cudaStream_t stream) {
-  // a single weight stack runs as two adjacent 16-row blocks of that stack
+  // A single weight stack runs as adjacent 16-row blocks of that stack: four per unit for
+  // routed tiles of one token set when the tile table's bound gives at least eight such
+  // units per SM (two 512-byte chunks per unit at K = 2048, where two blocks make every
+  // unit a single chunk and its per-unit work a larger share), two otherwise (fewer,
+  // larger units would leave the SMs unevenly loaded, and dense products need more units).
+  constexpr bool kWide = (BITS == 4 || BITS == 8) && GS * BITS / 8 <= 64;
+  if constexpr (kWide) {
+    const int64_t wide_units = a.max_tiles * ((a.N + 4 * kRows - 1) / (4 * kRows));
+    if (prm.pair && nt == 1 && a.dense_rows == 0 && wide_units >= 8 * sm_count())
+      return launch_cfg<BITS, GS, 4, 1>(prm, a, stream);
+  }
   return nt == 2 ? launch_cfg<BITS, GS, 2, 2>(prm, a, stream)
                  : launch_cfg<BITS, GS, 2, 1>(prm, a, stream);
 }
