@@ -200,7 +200,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 
   const int64_t KB_TOTAL = p.K / GS;
   const int64_t NCH = (KB_TOTAL + C::KB_PER_CHUNK - 1) / C::KB_PER_CHUNK;
-  const int unit_rows = p.pair ? NMAT * kRows : kRows;  // output channels per unit
+  // A unit's 16-row blocks: NMAT of one stack (pair), or NMAT/2 of each of two stacks (block
+  // m of the up stack for m < NMAT/2, of the gate stack for the rest).
+  constexpr int kHalf = NMAT / 2;
+  const int unit_rows = p.pair ? NMAT * kRows : kHalf * kRows;  // output channels per unit
+  auto blk_stack = [&](int m) { return p.pair ? 0 : m / kHalf; };
+  auto blk_row = [&](int m) { return kRows * (p.pair ? m : m % kHalf); };
   const int64_t NB = (p.N + unit_rows - 1) / unit_rows;
   const int64_t units = num_tiles<NT>(p) * NB;
   const int64_t u_begin = units * blockIdx.x / gridDim.x;
@@ -247,8 +252,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
           if (p.code3d) {
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
-              tma_load_3d(st + m * C::BOXES * 2048, &p.tmap[p.pair ? 0 : m], &full[stage], 0,
-                          static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)),
+              tma_load_3d(st + m * C::BOXES * 2048, &p.tmap[blk_stack(m)], &full[stage], 0,
+                          static_cast<int32_t>(row0 + blk_row(m)),
                           static_cast<int32_t>(ch * C::BOXES));
           } else {
             const int32_t xw = static_cast<int32_t>(ch * (C::CHUNK_ROW_BYTES / 4));
@@ -256,8 +261,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
               for (int bx = 0; bx < C::BOXES; ++bx)
-                tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[p.pair ? 0 : m], &full[stage],
-                            xw + bx * 32, static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
+                tma_load_2d(st + (m * C::BOXES + bx) * 2048, &p.tmap[blk_stack(m)], &full[stage],
+                            xw + bx * 32, static_cast<int32_t>(row0 + blk_row(m)));
           }
           if (p.sb_tma) {
             const int32_t xg = static_cast<int32_t>(ch * C::KB_PER_CHUNK);
@@ -266,8 +271,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
 #pragma unroll
               for (int arr = 0; arr < 2; ++arr)
                 tma_load_2d(st + C::CODE_BYTES + (m * 2 + arr) * kRows * C::KB_PER_CHUNK * 2,
-                            &p.tmap_sb[p.pair ? 0 : m][arr], &full[stage], xg,
-                            static_cast<int32_t>(row0 + (p.pair ? kRows * m : 0)));
+                            &p.tmap_sb[blk_stack(m)][arr], &full[stage], xg,
+                            static_cast<int32_t>(row0 + blk_row(m)));
           }
         }
         if (p.sb_tma) continue;
@@ -275,8 +280,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
         const int64_t kb0 = ch * C::KB_PER_CHUNK;
         const int ngroups = static_cast<int>(imin64(C::KB_PER_CHUNK, KB_TOTAL - kb0));
         const int pieces = ngroups * 2 / p.sb_vec;
-        // rows of each 16-row block inside [0, N): the tail block of a pair may be short
-        const int nrows = static_cast<int>(imin64(kRows, p.N - n0));
+        // rows of each 16-row block inside [0, N): a unit's tail blocks may be short
+        const int nrows = static_cast<int>(imin64(unit_rows, p.N - n0));
         const int tasks = NMAT * 2 * kRows * pieces;
         uint16_t* sb = reinterpret_cast<uint16_t*>(st + C::CODE_BYTES);
         for (int tk = lane; tk < tasks; tk += 32) {
@@ -284,9 +289,9 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
           const int rr = (tk / pieces) % kRows;
           const int arr = (tk / (pieces * kRows)) % 2;
           const int m = tk / (pieces * kRows * 2);
-          const int mrow = p.pair ? kRows * m + rr : rr;  // row inside the unit
-          if (mrow >= (p.pair ? static_cast<int>(imin64(NMAT * kRows, p.N - n0)) : nrows)) continue;
-          const int sm = p.pair ? 0 : m;  // the weight stack
+          const int mrow = blk_row(m) + rr;  // row inside the unit (of its stack)
+          if (mrow >= nrows) continue;
+          const int sm = blk_stack(m);  // the weight stack
           const uint16_t* src = (arr ? p.biases[sm] : p.scales[sm]) + (row0 + mrow) * KB_TOTAL + kb0;
           uint16_t* dst = sb + ((m * 2 + arr) * kRows + rr) * C::KB_PER_CHUNK;
           const int off = piece * (p.sb_vec / 2);
@@ -347,13 +352,15 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, NMAT, NT>::THREADS, 1)
             const int64_t n = n0 + kRows * m + row;
             if (n < p.N) yrow[n] = f32_to_bf16(v[m]);
           }
-        } else if (n0 + row < p.N) {
-          float out = v[0];
-          if constexpr (NMAT == 2) {
-            const float gte = v[1];
-            out = v[0] * (gte / (1.0f + expf(-gte)));
+        } else {
+#pragma unroll
+          for (int h = 0; h < kHalf; ++h) {  // up block h and gate block kHalf + h
+            const int64_t n = n0 + kRows * h + row;
+            if (n < p.N) {
+              const float gte = v[kHalf + h];
+              yrow[n] = f32_to_bf16(v[h] * (gte / (1.0f + expf(-gte))));
+            }
           }
-          yrow[n0 + row] = f32_to_bf16(out);
         }
       }
       __syncwarp();
@@ -706,15 +713,18 @@ cudaError_t launch_cfg(QmvParams prm, const GemmArgs& a, cudaStream_t stream) {
 
 template <int BITS, int GS>
 cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cudaStream_t stream) {
-  // A single weight stack runs as adjacent 16-row blocks of that stack: four per unit for
+  // A unit is four 16-row blocks (four of one stack, or two of each of up and gate) for
   // routed tiles of one token set when the tile table's bound gives at least eight such
-  // units per SM (two 512-byte chunks per unit at K = 2048, where two blocks make every
-  // unit a single chunk and its per-unit work a larger share), two otherwise (fewer,
-  // larger units would leave the SMs unevenly loaded, and dense products need more units).
+  // units per SM, else two (one of each stack, or two of one).  Four blocks spread each
+  // unit's fixed work -- the partial-sum hand-off, the next tile's row pointers, the
+  // activation fragments and group sums shared by the blocks -- over twice the weight
+  // bytes; fewer, larger units would leave the SMs unevenly loaded at small batches, and
+  // dense products need more units to fill the SMs.
   constexpr bool kWide = (BITS == 4 || BITS == 8) && GS * BITS / 8 <= 64;
   if constexpr (kWide) {
-    const int64_t wide_units = a.max_tiles * ((a.N + 4 * kRows - 1) / (4 * kRows));
-    if (prm.pair && nt == 1 && a.dense_rows == 0 && wide_units >= 8 * sm_count())
+    const int wide_rows = prm.pair ? 4 * kRows : 2 * kRows;  // channels of a four-block unit
+    const int64_t wide_units = a.max_tiles * ((a.N + wide_rows - 1) / wide_rows);
+    if (nt == 1 && a.dense_rows == 0 && wide_units >= 8 * sm_count())
       return launch_cfg<BITS, GS, 4, 1>(prm, a, stream);
   }
   return nt == 2 ? launch_cfg<BITS, GS, 2, 2>(prm, a, stream)
