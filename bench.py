@@ -47,12 +47,12 @@ LAYERS = 42
 M_CHAIN = 4
 
 # DRAM traffic of one fused up/gate launch over its algorithmic bytes, from an ncu
-# capture (dram__bytes_read.sum + dram__bytes_write.sum) of qmv_kernel<4,64,2,1> in this
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of qmv_kernel<4,64,4,1> in this
 # chain at 64 experts, layer 20 of the first warm-up step (28 touched experts:
-# 264,370,944 B read + 4,281,344 B written for 264,241,152 algorithmic bytes).
+# 264,368,384 B read + 3,879,424 B written for 264,241,152 algorithmic bytes).
 # The per-launch traffic reported below is this ratio times the launch's algorithmic
 # bytes (traffic scales with the experts touched).
-UPGATE_TRAFFIC_RATIO = (264_370_944 + 4_281_344) / 264_241_152
+UPGATE_TRAFFIC_RATIO = (264_368_384 + 3_879_424) / 264_241_152
 
 
 def matrix_bytes(N, K, group=GROUP, bits=BITS):

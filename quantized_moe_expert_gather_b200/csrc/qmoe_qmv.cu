@@ -11,8 +11,9 @@
 //
 // Structure (one persistent CTA per SM, 8 consumer warps + 1 producer warp + 1
 // epilogue warp):
-//   * the producer warp walks the CTA's contiguous range of (tile, 16-row block) units
-//     and, per K-chunk of 1 KB of each row (512 B with two token sets), loads each
+//   * the producer warp walks the CTA's contiguous range of units (a tile of routed rows
+//     and NMAT 16-row weight blocks: of the one stack, or half of each of two) and, per
+//     K-chunk of 1 KB of each row (512 B with two token sets or four blocks), loads each
 //     16-row block's packed codes with one 3-D TMA box (16 rows x 8 column blocks of
 //     128 B, 128B-swizzled so that the
 //     consumers' row-strided reads are free of bank conflicts; eight 2-D boxes of
