@@ -286,6 +286,22 @@ def _switch_oracle(x, idx, up, gate, down, group, bits):
     return O.switch_glu(x, remap, sel(up), sel(gate), sel(down))
 
 
+def test_switch_glu_decode_rows_bitwise_across_unit_shapes(gpu_lib, monkeypatch):
+    """A decode token's SwitchGLU output bits are the same in a 4-token call (the streaming
+    kernel's four-block units) as alone (two-block units): MTPLX PR #558, Summary (the
+    invariant lane); nuvec-core quantized.rs few_row_products_equal_one_row_products_bit_for_bit."""
+    q = gpu_lib
+    monkeypatch.setenv("QMOE_FORCE_KERNEL", "qmv")
+    up, gate, down = _decode_weights()
+    x, idx = decode_tokens(3, 4)
+    W = [qweight(*t, 64, 4) for t in (up, gate, down)]
+    together = host_bits16(q.qmoe_switch_glu(dev_bf16(x), dev_u32(idx), *W, mode=0))
+    for t in range(4):
+        alone = host_bits16(q.qmoe_switch_glu(dev_bf16(x[t:t + 1]), dev_u32(idx[t:t + 1]), *W,
+                                              mode=0))
+        assert np.array_equal(alone[0], together[t]), t
+
+
 @pytest.mark.parametrize("M", [1, 4])
 def test_switch_glu_decode_layer(gpu_lib, kernel, M):
     """Decode layer at full size: hidden 4096, intermediate 2048, E=288, top-8."""
