@@ -721,7 +721,9 @@ cudaError_t launch_bits_gs(const QmvParams& prm, const GemmArgs& a, int nt, cuda
   // activation fragments and group sums shared by the blocks -- over twice the weight
   // bytes; fewer, larger units would leave the SMs unevenly loaded at small batches, and
   // dense products need more units to fill the SMs.
-  constexpr bool kWide = (BITS == 4 || BITS == 8) && GS * BITS / 8 <= 64;
+  // (4-bit codes in groups of 64, the decode codec measured and tested with four blocks;
+  // the other codecs keep two)
+  constexpr bool kWide = BITS == 4 && GS == 64;
   if constexpr (kWide) {
     const int wide_rows = prm.pair ? 4 * kRows : 2 * kRows;  // channels of a four-block unit
     const int64_t wide_units = a.max_tiles * ((a.N + wide_rows - 1) / wide_rows);
