@@ -1,6 +1,6 @@
 """Expert-parallel MoE layer (``quantized_moe_expert_gather_b200.ep``).
 
-* Two gloo ranks on CPU: the layer's exchange (counts, dispatch of rows and expert numbers,
+* Two and four gloo ranks on CPU: the layer's exchange (counts, dispatch of rows and expert numbers,
   return of the outputs, reassembly in expert order) with the local steps done by the
   oracle.  Each rank's result equals, bit for bit, the single-process oracle layer on its
   own tokens with every expert (the same rounding points), so the dispatch and combine
@@ -73,12 +73,18 @@ def _global_weights():
     return [random_qweight(rng, E, n, k, GROUP, BITS) for n, k in ((I, H), (I, H), (H, I))]
 
 
-def _tokens(rank):
+def _token_count(rank, ws):
+    """Routed tokens of a rank: different on every rank; with four ranks, rank 2 has none."""
+    return 0 if (ws == 4 and rank == 2) else 5 + 2 * rank
+
+
+def _tokens(rank, ws):
     from inputs import normal_bf16
     rng = np.random.default_rng(100 + rank)
-    T = 5 + 2 * rank
+    T = _token_count(rank, ws)
     x = normal_bf16(rng, (T, H))
-    idx = np.stack([rng.choice(E, size=TOP_K, replace=False) for _ in range(T)]).astype(np.uint32)
+    idx = np.array([rng.choice(E, size=TOP_K, replace=False) for _ in range(T)],
+                   np.uint32).reshape(T, TOP_K)
     p = rng.random((T, TOP_K)).astype(np.float32)
     return x, idx, (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
 
@@ -110,18 +116,20 @@ def _rank_main(rank, ws, port, out):
     local = [(w[rank * el:(rank + 1) * el], s[rank * el:(rank + 1) * el],
               b[rank * el:(rank + 1) * el], GROUP, BITS) for (w, s, b) in weights]
     layer = ExpertParallelMoE(*local, num_experts=E, ops=OracleOps(O))
-    x, idx, sc = _tokens(rank)
+    x, idx, sc = _tokens(rank, ws)
     got = layer(_bf16(x), torch.from_numpy(idx.view(np.int32)), torch.from_numpy(sc))
-    want = _reference(O, x, idx, sc, weights)
+    want = _reference(O, x, idx, sc, weights) if x.shape[0] else np.zeros((0, H), np.uint16)
     order, _, off = O.sort_by_expert(idx.reshape(-1).astype(np.int64), E)
     out[rank] = (bool(np.array_equal(got.numpy(), want)), layer.split_counts(torch.from_numpy(off)),
-                 float(np.abs(got.numpy() - want).max()))
+                 float(np.abs(got.numpy() - want).max()) if want.size else 0.0)
     dist.barrier()
     dist.destroy_process_group()
 
 
-def test_expert_parallel_two_gloo_ranks_match_the_oracle_layer_bitwise():
-    ws = 2
+@pytest.mark.parametrize("ws", [2, 4])
+def test_expert_parallel_gloo_ranks_match_the_oracle_layer_bitwise(ws):
+    """Two ranks (four experts each), and four ranks (two each) of which one routes no
+    tokens but still serves its experts to the others."""
     with mp.Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(ws, _free_port(), out), nprocs=ws,
@@ -130,8 +138,7 @@ def test_expert_parallel_two_gloo_ranks_match_the_oracle_layer_bitwise():
     for rank in range(ws):
         equal, sends, err = got[rank]
         assert equal, f"rank {rank}: max |got - want| = {err}"
-        T = 5 + 2 * rank
-        assert sum(sends) == T * TOP_K  # every routed row sent to exactly one owner
+        assert sum(sends) == _token_count(rank, ws) * TOP_K  # each routed row to one owner
 
 
 @pytest.mark.gpu
@@ -144,7 +151,7 @@ def test_expert_parallel_layer_one_gpu(gpu_lib):
     W = [qweight(*w, GROUP, BITS) for w in weights]
     layer = ExpertParallelMoE(*W, num_experts=E)
     for rank in range(2):
-        x, idx, sc = _tokens(rank)
+        x, idx, sc = _tokens(rank, 1)
         got = layer(dev_bf16(x), dev_u32(idx), dev_f32(sc))
         torch.cuda.synchronize()
         assert_close(f"EP layer tokens {rank}", got, _reference(O, x, idx, sc, weights))
