@@ -14,10 +14,10 @@
 //   * the producer warp walks the CTA's contiguous range of units (a tile of routed rows
 //     and NMAT 16-row weight blocks: of the one stack, or half of each of two) and, per
 //     K-chunk of 1 KB of each row (512 B with two token sets or four blocks), loads each
-//     16-row block's packed codes with one 3-D TMA box (16 rows x 8 column blocks of
-//     128 B, 128B-swizzled so that the
-//     consumers' row-strided reads are free of bank conflicts; eight 2-D boxes of
-//     128 B x 16 rows when a row is not a whole number of column blocks) and the
+//     16-row block's packed codes with one 3-D TMA box (16 rows x 8 (or 4) column blocks
+//     of 128 B, 128B-swizzled so that the consumers' row-strided reads are free of bank
+//     conflicts; one 2-D box of 128 B x 16 rows per column block when a row is not a
+//     whole number of column blocks) and the
 //     matching scales/biases with 2-D TMA boxes (cp.async when their row pitch is not
 //     a multiple of 16 bytes), into a ring of stages guarded by full/empty mbarriers.
 //     Few large copies per stage matter: the TMA issue and mbarrier round trip of
