@@ -109,3 +109,25 @@ def test_workspace_sizes_grow_with_rows(lib):
     large = lib.qmoe_gather_qmm_workspace_size(4096, 1, 288, 2048, 4096)
     assert large > small > 0
     assert lib.qmoe_sort_by_expert_workspace_size(131072, 256) > lib.qmoe_sort_by_expert_workspace_size(8, 256)
+
+
+def test_gather_mm_and_ep_pack_reject_bad_arguments_on_host(lib):
+    fake = 1 << 20  # never dereferenced: validation fails first
+    # gather_mm: K a whole number of 64-k stages; workspace; 16-byte aligned operands
+    need = lib.qmoe_gather_mm_workspace_size(4, 1, 8, 16, 64)
+    assert need > 0
+    assert lib.qmoe_gather_mm(fake, 4, 1, 96, fake, 8, 16, None, fake, 4, 0, fake, need,
+                              fake, None, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_gather_mm(fake, 4, 1, 64, fake, 8, 16, None, fake, 4, 0, fake, need - 1,
+                              fake, None, None) == ERR_WORKSPACE
+    assert lib.qmoe_gather_mm(fake + 2, 4, 1, 64, fake, 8, 16, None, fake, 4, 0, fake, need,
+                              fake, None, None) == ERR_ARG
+    assert lib.qmoe_gather_mm(fake, 4, 1, 64, fake, 8, 16, None, fake, 0, 0, None, 0,
+                              fake, None, None) == 0  # no batches: nothing to do
+    # ep_pack: hidden size a multiple of 8, positive sizes, aligned rows; no rows is a no-op
+    assert lib.qmoe_ep_pack(fake, 2, 12, 2, fake, fake, 4, fake, fake, None, None) == ERR_UNSUPPORTED
+    assert lib.qmoe_ep_pack(fake, -1, 16, 2, fake, fake, 4, fake, fake, None, None) == ERR_ARG
+    assert lib.qmoe_ep_pack(fake, 2, 16, 2, fake, fake, 0, fake, fake, None, None) == ERR_ARG
+    assert lib.qmoe_ep_pack(fake + 2, 2, 16, 2, fake, fake, 4, fake, fake, None, None) == ERR_ARG
+    assert lib.qmoe_ep_pack(fake, 2, 16, 2, None, fake, 4, fake, fake, None, None) == ERR_ARG
+    assert lib.qmoe_ep_pack(None, 0, 16, 2, None, None, 4, None, None, None, None) == 0
